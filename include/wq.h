@@ -1,0 +1,143 @@
+/*
+ * wq.h -- C ABI of libwq.so: weight-only integer-quantised GEMM for NVIDIA
+ * B200 (sm_100a).
+ *
+ * Weights W (fp16, [N, K] row-major, the nn.Linear layout) are stored as b-bit
+ * integer codes (b = 2, 3, 4 or 8) on the uniform asymmetric min-max grid, one
+ * grid per row or per group of `group` consecutive input columns:
+ *
+ *   lo = min(0, min w), hi = max(0, max w)           over the row / group
+ *   scale = fp16_rne((hi - lo) / (2^b - 1))          (1.0 if that rounds to 0)
+ *   zero  = rint(-lo / scale)                        (0 when scale was 0)
+ *   q     = clamp(rint(w / scale) + zero, 0, 2^b - 1)   rint: half to even
+ *   w'    = scale * (q - zero)
+ *
+ * Sources: "OPTQ: Accurate Quantization for Generative Pre-trained
+ * Transformers" (reproducibility summary, row "Experiment Setup": uniform
+ * per-row asymmetric quantisation on the min-max grid); "Platform For AI:
+ * BladeLLM model quantization" (section "block_wise_quant": one parameter set
+ * per block of input channels; section "Quantization algorithms > MinMax":
+ * round to nearest, no calibration data).  The range always containing 0, the
+ * half-to-even rounding, the fp16 rounding of the scale and the degenerate
+ * scale rule are this library's readings of what those pages leave open.
+ *
+ * Packed code layout ("[Feature Request] 4bit and 2bit and 1bit quantization
+ * support", onnxruntime issue 14997: several low-bit codes per machine word):
+ * codes are uint32 [N, K*b/32] row-major, least-significant bits first along K.
+ *   b = 2, 4, 8: code k of a row is in word k/(32/b) at bit b*(k mod 32/b)
+ *                (16, 8, 4 codes per word);
+ *   b = 3:       the 32 codes of unit u = k/32 fill the 96-bit little-endian
+ *                value of words 3u, 3u+1, 3u+2; code j = k mod 32 sits at bit 3j
+ *                (codes 10 and 21 of each unit straddle two words).
+ * Scales and zeros are fp16 [N, G] row-major, G = K/group (G = 1 per row);
+ * every zero is a non-negative integer, exact in fp16.
+ *
+ * Common rules for the compute calls:
+ *   - every pointer is a DEVICE pointer on the current CUDA device, 16-byte
+ *     aligned; the caller allocates and owns every buffer, the library never
+ *     allocates, frees or keeps a pointer after the call returns;
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream); the work
+ *     is enqueued on it and the call returns without synchronising;
+ *   - `group` is 0 or K (one grid per row), or a multiple of 32 dividing K;
+ *   - K must be a multiple of 32; M, N, K >= 1;
+ *   - arguments are checked before anything is launched; on any non-OK status
+ *     nothing is launched and no output byte is written;
+ *   - WQ_ERR_CUDA reports a launch error (the CUDA error is left for
+ *     cudaGetLastError to read);
+ *   - W must be finite (not checked).
+ */
+#ifndef WQ_H
+#define WQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  WQ_OK = 0,
+  WQ_ERR_NULL = 1,                /* a required pointer is NULL */
+  WQ_ERR_BITS = 2,                /* bits not in {2, 3, 4, 8} */
+  WQ_ERR_GROUP = 3,               /* group not 0, K, or a multiple of 32 dividing K */
+  WQ_ERR_SHAPE = 4,               /* M, N or K < 1, K not a multiple of 32, or too large */
+  WQ_ERR_ALIGN = 5,               /* a pointer is not 16-byte aligned */
+  WQ_ERR_UNSUPPORTED_DEVICE = 6,  /* current device is not compute capability 10.0 */
+  WQ_ERR_CUDA = 7,                /* a CUDA runtime call or launch failed */
+  WQ_ERR_DEVICE_TIMEOUT = 8       /* a bounded device-side wait expired (see below) */
+} wq_status;
+
+/*
+ * wq_quantize_rtn -- round-to-nearest quantisation and packing of W.
+ * (Grid: OPTQ page, "Experiment Setup"; groups: BladeLLM page,
+ * "block_wise_quant"; rounding: BladeLLM page, "Quantization algorithms >
+ * MinMax".)
+ *
+ *   W_f16      in   fp16 [N, K] row-major
+ *   N, K            rows (outputs) and columns (inputs)
+ *   bits            2, 3, 4 or 8
+ *   group           0 or K (per row), or a multiple of 32 dividing K
+ *   codes      out  uint32 [N, wq_codes_words(N, K, bits) / N], layout above
+ *   scales_f16 out  fp16 [N, G]
+ *   zeros_f16  out  fp16 [N, G]
+ *   stream          cudaStream_t
+ *
+ * Results are bit-exact: codes, scales and zeros are the unique values the
+ * grid definition above gives (fp64 scale rounding, IEEE fp32 division and
+ * half-to-even rint for zero and codes).
+ */
+wq_status wq_quantize_rtn(const void* W_f16, int64_t N, int64_t K, int bits, int64_t group,
+                          uint32_t* codes, void* scales_f16, void* zeros_f16, void* stream);
+
+/*
+ * wq_gemm -- y = x . W'^T with W' dequantised on the fly from the codes.
+ * (Dequantise-in-the-matmul: onnxruntime issue 14997, weights kept in 4 bit and
+ * converted to float when used; BladeLLM page, "Background information >
+ * Solutions" and "Quantization modes > weight_only_quant": low-bit weights cut
+ * the bytes moved from GPU memory, the bound in memory-limited decoding.)
+ *
+ *   x_bf16     in   bf16 [M, K] row-major
+ *   M, N, K         batch rows, output features, input features
+ *   codes      in   packed codes as written by wq_quantize_rtn
+ *   scales_f16 in   fp16 [N, G]
+ *   zeros_f16  in   fp16 [N, G]
+ *   bits, group     as given to wq_quantize_rtn
+ *   y_bf16     out  bf16 [M, N] row-major; must not overlap the inputs
+ *   stream          cudaStream_t
+ *
+ * Products and sums are fp32; y is rounded once to bf16 (RNE).  M <= 16 runs a
+ * CUDA-core GEMV (codes streamed once with wide loads, unpacked in registers);
+ * larger M runs a tensor-core GEMM (tcgen05 MMA, operands staged by TMA, W'
+ * dequantised to bf16 in shared memory, accumulators in tensor memory).  Each
+ * y element is within 2e-3 * sum_k |x w'| + 1e-3 of the exact fp64 value.
+ */
+wq_status wq_gemm(const void* x_bf16, int64_t M, int64_t N, int64_t K, const uint32_t* codes,
+                  const void* scales_f16, const void* zeros_f16, int bits, int64_t group,
+                  void* y_bf16, void* stream);
+
+/* Number of uint32 words of packed codes for an [N, K] matrix: N*K*bits/32
+ * (0 if bits or K are invalid). */
+size_t wq_codes_words(int64_t N, int64_t K, int bits);
+
+/* Number of fp16 scales (and of zeros): N * G, G = K/group or 1 per row
+ * (0 if group or K are invalid). */
+size_t wq_params_count(int64_t N, int64_t K, int64_t group);
+
+/* Static, NUL-terminated description of a status code. */
+const char* wq_status_string(wq_status status);
+
+/*
+ * wq_last_device_error -- WQ_ERR_DEVICE_TIMEOUT if, since the previous call, a
+ * kernel on the current device gave up a bounded wait (a pipeline barrier that
+ * never completed); WQ_OK otherwise.  Synchronises the device and clears the
+ * flag.  A kernel that gives up leaves its outputs undefined but the CUDA
+ * context usable.
+ */
+wq_status wq_last_device_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WQ_H */

@@ -1,0 +1,529 @@
+// gemm_tc.cu -- prefill y = x . W'^T on the Blackwell tensor cores (tcgen05).
+//
+// Dequantise inside the matmul ("[Feature Request] 4bit and 2bit and 1bit
+// quantization support": weights stay packed and become floats on the GPU;
+// "Platform For AI: BladeLLM model quantization", "Background information >
+// Solutions").  For a batch of hundreds of rows the product is a dense
+// contraction, so it runs on the tensor cores with W' rebuilt in bf16 on chip.
+//
+// One CTA computes a 256 x 256 tile of y (256 batch rows x 256 output
+// features) over the whole K, in 64-wide K steps:
+//   warp 0      TMA producer: x tiles (bf16, 128-byte swizzled, 256 x 64) and
+//               packed code tiles (256 rows x 128 codes, unswizzled) into two
+//               shared-memory rings;
+//   warp 1      owns tensor memory (512 columns: two 128 x 256 fp32
+//               accumulators) and one lane issues the MMAs:
+//               tcgen05.mma.cta_group::1.kind::f16, M = 128, N = 256, K = 16,
+//               bf16 x bf16 -> fp32, A = x (two 128-row halves), B = W';
+//   warps 2..9  dequantise: codes -> w' = bf16_rne(scale * (q - zero)) (the
+//               product is exact in fp32, so w' is rounded once) written in the
+//               canonical K-major 128-byte-swizzled layout the MMA reads, then
+//               the epilogue: tcgen05.ld of the accumulators -> bf16 -> y.
+// With one grid per row the scale is constant along K, so the MMA is fed the
+// exact integers q - zero (exact in bf16 up to 256 in magnitude) and the fp32
+// scale of each output column is applied in the epilogue: the products are
+// then exact, as in the GEMV.  (Rounding scale * (q - zero) to bf16 would give
+// every weight of a row the same relative error, which does not average out.)
+// Stage hand-offs use mbarriers; tcgen05.commit frees a stage when the MMAs
+// that read it have completed.  Every wait is bounded in time: a wait that
+// expires raises a device flag (read by wq_last_device_error), makes the CTA
+// stop, drain its copies in flight and free its tensor memory.
+#include <cuda.h>   // CUtensorMap types only; the driver entry point is fetched at run time
+
+#include "wq_internal.cuh"
+
+namespace wq {
+
+// Set by a kernel that gave up a bounded wait; read and cleared by the host.
+__device__ unsigned int g_timeout_flag;
+
+namespace {
+
+constexpr int BM = 256, BN = 256, BK = 64, CK = 128;
+constexpr int kMmaM = 128, kMmaN = 256, kMmaK = 16;
+constexpr int kDqWarps = 8;
+constexpr int kThreads = 64 + 32 * kDqWarps;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kABytes = BM * BK * 2;
+constexpr uint32_t kBBytes = BN * BK * 2;
+constexpr uint64_t kWaitNs = 1000000000ull;      // 1 s: far beyond any healthy wait
+constexpr uint64_t kDrainNs = 200000000ull;      // 0.2 s for the exit path
+
+template <int BITS>
+struct TcCfg {
+  static constexpr int kStages = BITS == 8 ? 2 : 3;        // x / W' ring
+  static constexpr int kCStages = 2;                       // codes ring (128 K each)
+  static constexpr uint32_t kCBytes = uint32_t(BN) * CK * BITS / 8;
+  static constexpr uint32_t kRingBytes = kStages * (kABytes + kBBytes) + kCStages * kCBytes;
+  static constexpr uint32_t kSmem = kRingBytes + 1024 + 256 + 4 * BN;
+};
+static_assert(TcCfg<4>::kSmem <= 232448, "shared memory");
+static_assert(TcCfg<8>::kSmem <= 232448, "shared memory");
+static_assert(TcCfg<3>::kSmem <= 232448, "shared memory");
+
+// ------------------------------------------------------------------ PTX
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint64_t* b, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(b)), "r"(count));
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* b) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(b)) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* b, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(b)),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* b, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(b)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Bounded wait.  Returns false if the CTA has aborted or the wait expired (the
+// latter raises the CTA abort word and the device flag).
+__device__ __noinline__ bool mbar_wait(uint64_t* b, uint32_t parity, volatile uint32_t* abort) {
+  if (mbar_try_wait(b, parity)) return true;
+  const uint64_t t0 = global_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(b, parity)) return true;
+    if ((i & 63u) == 0) {
+      if (*abort) return false;
+      if (global_ns() - t0 > kWaitNs) {
+        *abort = 1u;
+        atomicExch(&g_timeout_flag, 1u);
+        return false;
+      }
+    }
+  }
+}
+// Exit-path wait for copies still in flight: ignores the abort word.
+__device__ __noinline__ void mbar_drain(uint64_t* b, uint32_t parity) {
+  const uint64_t t0 = global_ns();
+  while (!mbar_try_wait(b, parity)) {
+    if (global_ns() - t0 > kDrainNs) {
+      atomicExch(&g_timeout_flag, 1u);
+      return;
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                            int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
+// 1024 bytes apart (SBO), sm_100 descriptor version 1.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= uint64_t((saddr & 0x3FFFFu) >> 4);
+  d |= uint64_t(16u >> 4) << 16;
+  d |= uint64_t(1024u >> 4) << 32;
+  d |= uint64_t(1) << 46;
+  d |= uint64_t(2) << 61;
+  return d;
+}
+
+// Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, both
+// K-major, N = 256, M = 128.
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(kMmaN >> 3) << 17) |
+                            (uint32_t(kMmaM >> 4) << 24);
+
+__device__ __forceinline__ void umma(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t accum) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(kIdesc), "r"(accum));
+}
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Code i (0..31) of a 32-code unit (layout of include/wq.h).
+template <int BITS>
+__device__ __forceinline__ uint32_t unit_code(const uint32_t (&w)[BITS], int i) {
+  if constexpr (BITS == 3) {
+    const int bit = 3 * i, a = bit >> 5, sh = bit & 31;
+    const uint32_t nxt = (a + 1 < 3) ? w[(a + 1) % 3] : 0u;
+    return __funnelshift_r(w[a], nxt, sh) & 7u;
+  } else {
+    constexpr int per = 32 / BITS;
+    return (w[i / per] >> (BITS * (i % per))) & ((1u << BITS) - 1u);
+  }
+}
+
+template <int BITS>
+__device__ __forceinline__ void lds_unit(const uint8_t* p, uint32_t (&w)[BITS]) {
+  if constexpr (BITS == 2) {
+    const uint2 v = *reinterpret_cast<const uint2*>(p);
+    w[0] = v.x; w[1] = v.y;
+  } else if constexpr (BITS == 4) {
+    const uint4 v = *reinterpret_cast<const uint4*>(p);
+    w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
+  } else if constexpr (BITS == 8) {
+    const uint4 a = reinterpret_cast<const uint4*>(p)[0];
+    const uint4 b = reinterpret_cast<const uint4*>(p)[1];
+    w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
+    w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
+  } else {
+    const uint32_t* q = reinterpret_cast<const uint32_t*>(p);
+    w[0] = q[0]; w[1] = q[1]; w[2] = q[2];
+  }
+}
+
+__device__ __forceinline__ uint32_t bf162_bits(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);   // a -> low half (lower address)
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+template <int BITS>
+__global__ void __launch_bounds__(kThreads, 1)
+gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_c,
+               const __half* __restrict__ scales, const __half* __restrict__ zeros, int64_t M,
+               int64_t N, int64_t K, int64_t g, FastDiv units_per_group,
+               __nv_bfloat16* __restrict__ y) {
+  using Cfg = TcCfg<BITS>;
+  constexpr int S = Cfg::kStages, SC = Cfg::kCStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = base;                                   // [S][256 x 64 bf16], swizzled
+  uint8_t* sB = sA + S * kABytes;                       // [S][256 x 64 bf16], swizzled
+  uint8_t* sC = sB + S * kBBytes;                       // [SC][256 x 128 codes]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sC + SC * Cfg::kCBytes);
+  uint64_t* full_a = bars;             // TMA x landed            (1 arrival + bytes)
+  uint64_t* full_b = full_a + S;       // W' written             (kDqWarps arrivals)
+  uint64_t* empty_ab = full_b + S;     // MMAs done with stage   (commit)
+  uint64_t* full_c = empty_ab + S;     // TMA codes landed       (1 arrival + bytes)
+  uint64_t* empty_c = full_c + SC;     // codes consumed         (kDqWarps arrivals)
+  uint64_t* tmem_full = empty_c + SC;  // accumulators final     (commit)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tmem_full + 1);
+  volatile uint32_t* abort = tmem_slot + 1;
+
+  float* col_scale = reinterpret_cast<float*>(tmem_slot + 2);   // [BN], per-row grids only
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t n0 = int64_t(blockIdx.x) * BN, m0 = int64_t(blockIdx.y) * BM;
+  const int KT = int((K + BK - 1) / BK);
+  const bool rowwise = (g == K);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full_a[s], 1);
+      mbar_init(&full_b[s], kDqWarps);
+      mbar_init(&empty_ab[s], 1);
+    }
+    for (int s = 0; s < SC; ++s) {
+      mbar_init(&full_c[s], 1);
+      mbar_init(&empty_c[s], kDqWarps);
+    }
+    mbar_init(tmem_full, 1);
+    *abort = 0u;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(kTmemCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int issued_a = 0, issued_c = 0;
+      bool ok = true;
+      for (int kt = 0; kt < KT && ok; ++kt) {
+        if ((kt & 1) == 0) {                            // codes for K [kt*64, kt*64 + 128)
+          const int c = kt >> 1, cs = c % SC;
+          if (c >= SC) ok = mbar_wait(&empty_c[cs], ((c / SC) - 1) & 1, abort);
+          if (!ok) break;
+          mbar_expect_tx(&full_c[cs], Cfg::kCBytes);
+          tma_load_2d(sC + cs * Cfg::kCBytes, &tm_c, &full_c[cs], c * (CK * BITS / 32), int(n0));
+          ++issued_c;
+        }
+        const int s = kt % S;
+        if (kt >= S) ok = mbar_wait(&empty_ab[s], ((kt / S) - 1) & 1, abort);
+        if (!ok) break;
+        mbar_expect_tx(&full_a[s], kABytes);
+        tma_load_2d(sA + s * kABytes, &tm_x, &full_a[s], kt * BK, int(m0));
+        ++issued_a;
+      }
+      if (!ok) {   // let the copies still in flight land before shared memory goes away
+        for (int kt = (issued_a > S ? issued_a - S : 0); kt < issued_a; ++kt)
+          mbar_drain(&full_a[kt % S], (kt / S) & 1);
+        for (int c = (issued_c > SC ? issued_c - SC : 0); c < issued_c; ++c)
+          mbar_drain(&full_c[c % SC], (c / SC) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      bool ok = true;
+      for (int kt = 0; kt < KT && ok; ++kt) {
+        const int s = kt % S;
+        const uint32_t par = (kt / S) & 1;
+        ok = mbar_wait(&full_a[s], par, abort) && mbar_wait(&full_b[s], par, abort);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t a0 = smem_u32(sA + s * kABytes);
+        const uint32_t b0 = smem_u32(sB + s * kBBytes);
+#pragma unroll
+        for (int kk = 0; kk < BK / kMmaK; ++kk) {
+          const uint64_t bd = sw128_desc(b0 + kk * kMmaK * 2);
+#pragma unroll
+          for (int mt = 0; mt < BM / kMmaM; ++mt) {
+            const uint64_t ad = sw128_desc(a0 + mt * (kMmaM * 128) + kk * kMmaK * 2);
+            umma(tmem + uint32_t(mt * kMmaN), ad, bd, (kt > 0 || kk > 0) ? 1u : 0u);
+          }
+        }
+        umma_commit(&empty_ab[s]);
+      }
+      umma_commit(tmem_full);      // always: the teardown waits on it before freeing TMEM
+    }
+  } else {
+    // ------------------------------------------------------------ dequantise
+    const int dw = warp - 2;
+    const int cu = lane & 1;                 // 32-code unit within the 64-wide K step
+    const int64_t G = K / g;
+    if (rowwise) {                           // epilogue scale of each output column
+      const int c = threadIdx.x - 64;
+      col_scale[c] = (n0 + c < N) ? __half2float(scales[(n0 + c) * G]) : 0.0f;
+      asm volatile("bar.sync 1, %0;" ::"n"(32 * kDqWarps) : "memory");
+    }
+    bool ok = true;
+    for (int kt = 0; kt < KT && ok; ++kt) {
+      const int c = kt >> 1, cs = c % SC, s = kt % S;
+      ok = mbar_wait(&full_c[cs], (c / SC) & 1, abort);
+      if (ok && kt >= S) ok = mbar_wait(&empty_ab[s], ((kt / S) - 1) & 1, abort);
+      ok = __all_sync(0xffffffffu, ok);      // the warp leaves the loop together
+      if (!ok) break;
+      const uint8_t* ctile = sC + cs * Cfg::kCBytes;
+      uint8_t* btile = sB + s * kBBytes;
+      const int64_t k = int64_t(kt) * BK + 32 * cu;
+      const int ucode = (kt & 1) * 2 + cu;   // unit index within the 128-code stage
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const int r = 32 * dw + (lane >> 1) + 16 * i;
+        const int64_t n = n0 + r;
+        float sc = 0.0f, zb = 8388608.0f;
+        if (n < N && k < K) {
+          const uint32_t grp = units_per_group.div(uint32_t(k >> 5));
+          sc = rowwise ? 1.0f : __half2float(scales[n * G + grp]);
+          zb = 8388608.0f + __half2float(zeros[n * G + grp]);
+        }
+        uint32_t w[BITS];
+        lds_unit<BITS>(ctile + r * (CK * BITS / 8) + ucode * (4 * BITS), w);
+        uint8_t* brow = btile + r * 128;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          uint32_t p[4];
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const int i0 = 8 * j + 2 * t;
+            const float a = (__int_as_float(0x4B000000 | int(unit_code<BITS>(w, i0))) - zb) * sc;
+            const float b = (__int_as_float(0x4B000000 | int(unit_code<BITS>(w, i0 + 1))) - zb) * sc;
+            p[t] = bf162_bits(a, b);
+          }
+          const int chunk = (cu * 4 + j) ^ (r & 7);
+          *reinterpret_cast<uint4*>(brow + chunk * 16) = make_uint4(p[0], p[1], p[2], p[3]);
+        }
+      }
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&full_b[s]);
+        if (kt & 1 || kt == KT - 1) mbar_arrive(&empty_c[cs]);
+      }
+    }
+    // ------------------------------------------------------------ epilogue
+    if (ok) ok = mbar_wait(tmem_full, 0, abort);
+    ok = __all_sync(0xffffffffu, ok);        // tcgen05.ld needs the whole warp
+    if (ok) {
+      tc_fence_after();
+      const int q = warp & 3;                  // TMEM lane quarter this warp may access
+      const int mt = dw >> 2;
+      const int64_t m = m0 + mt * kMmaM + 32 * q + lane;
+      const bool vec = (N % 8) == 0;
+      for (int cb = 0; cb < kMmaN / 32; ++cb) {
+        uint32_t r[32];
+        tmem_ld32(tmem + (uint32_t(32 * q) << 16) + uint32_t(mt * kMmaN + cb * 32), r);
+        if (rowwise) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            r[j] = __float_as_uint(__uint_as_float(r[j]) * col_scale[cb * 32 + j]);
+        }
+        const int64_t n = n0 + cb * 32;
+        if (m < M && n < N) {
+          __nv_bfloat16* dst = y + m * N + n;
+          if (vec && n + 32 <= N) {
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              uint4 o;
+              o.x = bf162_bits(__uint_as_float(r[8 * v + 0]), __uint_as_float(r[8 * v + 1]));
+              o.y = bf162_bits(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3]));
+              o.z = bf162_bits(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5]));
+              o.w = bf162_bits(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7]));
+              reinterpret_cast<uint4*>(dst)[v] = o;
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (n + j < N) dst[j] = __float2bfloat16_rn(__uint_as_float(r[j]));
+          }
+        }
+      }
+    }
+  }
+
+  // ------------------------------------------------------------ teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    if (*abort) {
+      if (lane == 0) mbar_drain(tmem_full, 0);   // MMAs issued must finish before TMEM is freed
+      __syncwarp();
+    }
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
+  }
+}
+
+// ------------------------------------------------------------------ host
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<EncodeTiledFn>(nullptr);
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+template <int BITS>
+cudaError_t launch_bits(const __nv_bfloat16* x, int64_t M, int64_t N, int64_t K,
+                        const uint32_t* codes, const __half* scales, const __half* zeros,
+                        int64_t g, __nv_bfloat16* y, cudaStream_t st) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return cudaErrorNotSupported;
+  CUtensorMap tx, tc;
+  {
+    const cuuint64_t dims[2] = {cuuint64_t(K), cuuint64_t(M)};
+    const cuuint64_t strides[1] = {cuuint64_t(K) * 2};
+    const cuuint32_t box[2] = {BK, BM};
+    const cuuint32_t es[2] = {1, 1};
+    if (enc(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<__nv_bfloat16*>(x), dims, strides,
+            box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  {
+    const cuuint64_t dims[2] = {cuuint64_t(K * BITS / 32), cuuint64_t(N)};
+    const cuuint64_t strides[1] = {cuuint64_t(K * BITS / 8)};
+    const cuuint32_t box[2] = {CK * BITS / 32, BN};
+    const cuuint32_t es[2] = {1, 1};
+    if (enc(&tc, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(codes), dims, strides,
+            box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  constexpr uint32_t smem = TcCfg<BITS>::kSmem;
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BITS>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  const dim3 grid(unsigned((N + BN - 1) / BN), unsigned((M + BM - 1) / BM));
+  gemm_tc_kernel<BITS><<<grid, kThreads, smem, st>>>(tx, tc, scales, zeros, M, N, K, g,
+                                                      FastDiv(uint32_t(g / 32)), y);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool gemm_tc_supported(int64_t K, int bits) {
+  (void)bits;
+  return K % CK == 0;
+}
+
+cudaError_t launch_gemm_tc(const __nv_bfloat16* x, int64_t M, int64_t N, int64_t K,
+                           const uint32_t* codes, const __half* scales, const __half* zeros,
+                           int bits, int64_t g, __nv_bfloat16* y, cudaStream_t st) {
+  switch (bits) {
+    case 2: return launch_bits<2>(x, M, N, K, codes, scales, zeros, g, y, st);
+    case 3: return launch_bits<3>(x, M, N, K, codes, scales, zeros, g, y, st);
+    case 4: return launch_bits<4>(x, M, N, K, codes, scales, zeros, g, y, st);
+    default: return launch_bits<8>(x, M, N, K, codes, scales, zeros, g, y, st);
+  }
+}
+
+bool read_and_clear_timeout_flag(cudaError_t* err) {
+  unsigned int v = 0;
+  const unsigned int zero = 0;
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e == cudaSuccess) e = cudaMemcpyFromSymbol(&v, g_timeout_flag, sizeof(v));
+  if (e == cudaSuccess && v) e = cudaMemcpyToSymbol(g_timeout_flag, &zero, sizeof(zero));
+  *err = e;
+  return v != 0;
+}
+
+}  // namespace wq

@@ -1,0 +1,133 @@
+// wq_api.cu -- the C ABI of libwq.so (include/wq.h): argument checks, device
+// check, dispatch on the batch size, status strings.
+//
+// Every check runs before any launch, so a failing call writes nothing.
+#include <mutex>
+
+#include "../../include/wq.h"
+#include "wq_internal.cuh"
+
+namespace {
+
+bool valid_bits(int b) { return b == 2 || b == 3 || b == 4 || b == 8; }
+
+// K is assumed already checked (>= 32, multiple of 32).
+bool valid_group(int64_t K, int64_t group) {
+  if (group == 0 || group == K) return true;
+  return group > 0 && group % 32 == 0 && K % group == 0;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+constexpr int64_t kMaxDim = int64_t(1) << 31;
+
+// Compute capability of every device, checked once per device.
+wq_status check_device() {
+  static std::mutex mu;
+  static int verdict[64];   // 0 unknown, 1 ok, 2 unsupported
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return WQ_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return WQ_ERR_UNSUPPORTED_DEVICE;
+  std::lock_guard<std::mutex> lock(mu);
+  if (verdict[dev] == 0) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return WQ_ERR_CUDA;
+    verdict[dev] = (major == 10 && minor == 0) ? 1 : 2;
+  }
+  return verdict[dev] == 1 ? WQ_OK : WQ_ERR_UNSUPPORTED_DEVICE;
+}
+
+wq_status check_common(int64_t N, int64_t K, int bits, int64_t group) {
+  if (!valid_bits(bits)) return WQ_ERR_BITS;
+  if (N < 1 || K < 1 || K % 32 != 0 || N >= kMaxDim || K >= kMaxDim) return WQ_ERR_SHAPE;
+  if (!valid_group(K, group)) return WQ_ERR_GROUP;
+  return WQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t wq_codes_words(int64_t N, int64_t K, int bits) {
+  if (!valid_bits(bits) || N < 1 || K < 1 || K % 32 != 0) return 0;
+  return size_t(N) * size_t(K / 32) * size_t(bits);
+}
+
+size_t wq_params_count(int64_t N, int64_t K, int64_t group) {
+  if (N < 1 || K < 1 || K % 32 != 0 || !valid_group(K, group)) return 0;
+  return size_t(N) * size_t(K / wq::effective_group(K, group));
+}
+
+const char* wq_status_string(wq_status s) {
+  switch (s) {
+    case WQ_OK: return "ok";
+    case WQ_ERR_NULL: return "a required pointer is NULL";
+    case WQ_ERR_BITS: return "bits must be 2, 3, 4 or 8";
+    case WQ_ERR_GROUP: return "group must be 0, K, or a multiple of 32 that divides K";
+    case WQ_ERR_SHAPE: return "M, N, K must be >= 1 and < 2^31, K a multiple of 32";
+    case WQ_ERR_ALIGN: return "every pointer must be 16-byte aligned";
+    case WQ_ERR_UNSUPPORTED_DEVICE: return "the current device is not compute capability 10.0 (B200)";
+    case WQ_ERR_CUDA: return "a CUDA call or kernel launch failed";
+    case WQ_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait expired";
+  }
+  return "unknown status";
+}
+
+wq_status wq_quantize_rtn(const void* W_f16, int64_t N, int64_t K, int bits, int64_t group,
+                          uint32_t* codes, void* scales_f16, void* zeros_f16, void* stream) {
+  if (!W_f16 || !codes || !scales_f16 || !zeros_f16) return WQ_ERR_NULL;
+  wq_status st = check_common(N, K, bits, group);
+  if (st != WQ_OK) return st;
+  if (!aligned16(W_f16) || !aligned16(codes) || !aligned16(scales_f16) || !aligned16(zeros_f16))
+    return WQ_ERR_ALIGN;
+  if ((st = check_device()) != WQ_OK) return st;
+  cudaError_t e = wq::launch_quantize(static_cast<const __half*>(W_f16), N, K, bits,
+                                      wq::effective_group(K, group), codes,
+                                      static_cast<__half*>(scales_f16),
+                                      static_cast<__half*>(zeros_f16),
+                                      static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? WQ_OK : WQ_ERR_CUDA;
+}
+
+wq_status wq_gemm(const void* x_bf16, int64_t M, int64_t N, int64_t K, const uint32_t* codes,
+                  const void* scales_f16, const void* zeros_f16, int bits, int64_t group,
+                  void* y_bf16, void* stream) {
+  if (!x_bf16 || !codes || !scales_f16 || !zeros_f16 || !y_bf16) return WQ_ERR_NULL;
+  wq_status st = check_common(N, K, bits, group);
+  if (st != WQ_OK) return st;
+  if (M < 1 || M >= kMaxDim) return WQ_ERR_SHAPE;
+  if (!aligned16(x_bf16) || !aligned16(codes) || !aligned16(scales_f16) ||
+      !aligned16(zeros_f16) || !aligned16(y_bf16))
+    return WQ_ERR_ALIGN;
+  if ((st = check_device()) != WQ_OK) return st;
+  const int64_t g = wq::effective_group(K, group);
+  const auto* x = static_cast<const __nv_bfloat16*>(x_bf16);
+  const auto* s = static_cast<const __half*>(scales_f16);
+  const auto* z = static_cast<const __half*>(zeros_f16);
+  auto* y = static_cast<__nv_bfloat16*>(y_bf16);
+  auto strm = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (M > wq::kGemvMaxM && wq::gemm_tc_supported(K, bits)) {
+    e = wq::launch_gemm_tc(x, M, N, K, codes, s, z, bits, g, y, strm);
+  } else {
+    // Small batches, and K that the tensor-core path cannot stage with TMA
+    // (K not a multiple of 128): the GEMV, 16 batch rows per launch.
+    e = cudaSuccess;
+    for (int64_t m0 = 0; m0 < M && e == cudaSuccess; m0 += wq::kGemvMaxM) {
+      const int mc = int(M - m0 < wq::kGemvMaxM ? M - m0 : wq::kGemvMaxM);
+      e = wq::launch_gemv(x + m0 * K, mc, N, K, codes, s, z, bits, g, y + m0 * N, strm);
+    }
+  }
+  return e == cudaSuccess ? WQ_OK : WQ_ERR_CUDA;
+}
+
+wq_status wq_last_device_error(void) {
+  cudaError_t e = cudaSuccess;
+  const bool hit = wq::read_and_clear_timeout_flag(&e);
+  if (e != cudaSuccess) return WQ_ERR_CUDA;
+  return hit ? WQ_ERR_DEVICE_TIMEOUT : WQ_OK;
+}
+
+}  // extern "C"

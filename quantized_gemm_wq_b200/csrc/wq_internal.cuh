@@ -1,0 +1,53 @@
+// wq_internal.cuh -- declarations shared by the translation units of libwq.so.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace wq {
+
+// Largest M served by the CUDA-core GEMV; larger batches use the tensor cores.
+constexpr int kGemvMaxM = 16;
+
+// Effective group length: K for a per-row grid (group 0 or K).
+inline int64_t effective_group(int64_t K, int64_t group) { return (group == 0) ? K : group; }
+
+// Division of non-negative 32-bit n (< 2^31) by a fixed divisor d >= 1 with a
+// multiply-high and a shift (division by invariant integers using
+// multiplication, Granlund & Montgomery 1994): l = ceil(log2 d),
+// m = floor(2^32 (2^l - d) / d) + 1, n / d = (mulhi(n, m) + n) >> l.
+struct FastDiv {
+  uint32_t m = 1, l = 0;
+  FastDiv() = default;
+  explicit FastDiv(uint32_t d) {
+    l = 0;
+    while ((uint64_t(1) << l) < d) ++l;
+    m = uint32_t(((uint64_t(1) << 32) * ((uint64_t(1) << l) - d)) / d + 1);
+  }
+  __device__ __forceinline__ uint32_t div(uint32_t n) const {
+    return uint32_t((uint64_t(__umulhi(n, m)) + n) >> l);
+  }
+};
+
+// ---- launchers (arguments already validated by the C ABI layer) ----------
+cudaError_t launch_quantize(const __half* W, int64_t N, int64_t K, int bits, int64_t g,
+                            uint32_t* codes, __half* scales, __half* zeros, cudaStream_t st);
+
+cudaError_t launch_gemv(const __nv_bfloat16* x, int M, int64_t N, int64_t K,
+                        const uint32_t* codes, const __half* scales, const __half* zeros,
+                        int bits, int64_t g, __nv_bfloat16* y, cudaStream_t st);
+
+// True when the tensor-core path can stage this K with TMA (K a multiple of 128).
+bool gemm_tc_supported(int64_t K, int bits);
+
+cudaError_t launch_gemm_tc(const __nv_bfloat16* x, int64_t M, int64_t N, int64_t K,
+                           const uint32_t* codes, const __half* scales, const __half* zeros,
+                           int bits, int64_t g, __nv_bfloat16* y, cudaStream_t st);
+
+// Reads and clears the device-side "bounded wait expired" flag of the current
+// device (synchronises the device).  Returns true if it was set.
+bool read_and_clear_timeout_flag(cudaError_t* err);
+
+}  // namespace wq

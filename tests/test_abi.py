@@ -1,0 +1,64 @@
+"""The C-ABI library loads on a host without a GPU, exports every function
+include/wq.h declares, and rejects bad arguments before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def wq():
+    import quantized_gemm_wq_b200 as wq
+    return wq
+
+
+def _declared_functions():
+    src = open(os.path.join(ROOT, "include", "wq.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(wq_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_exports_every_declared_function(wq):
+    names = _declared_functions()
+    assert set(names) == set(wq.EXPORTED)
+    for n in names:
+        assert hasattr(wq.lib, n), n
+
+
+def test_layout_helpers(wq):
+    assert wq.wq_codes_words(4096, 4096, 4) == 4096 * 4096 * 4 // 32
+    assert wq.wq_codes_words(3, 96, 3) == 3 * 9
+    assert wq.wq_codes_words(3, 40, 3) == 0
+    assert wq.wq_codes_words(3, 64, 5) == 0
+    assert wq.wq_params_count(4096, 4096, 128) == 4096 * 32
+    assert wq.wq_params_count(5, 4096, 0) == 5
+    assert wq.wq_params_count(5, 4096, 4096) == 5
+    assert wq.wq_params_count(5, 4096, 48) == 0
+
+
+def test_status_strings(wq):
+    for s in range(9):
+        assert len(wq.wq_status_string(s)) >= 2
+    assert "unknown" in wq.wq_status_string(99)
+
+
+def test_rejects_before_device(wq):
+    L = wq.lib
+    P = 1 << 20          # a non-null, 16-byte aligned fake address: never dereferenced
+    q = L.wq_quantize_rtn
+    assert q(None, 4, 64, 4, 32, P, P, P, None) == wq.WQ_ERR_NULL
+    assert q(P, 4, 64, 5, 32, P, P, P, None) == wq.WQ_ERR_BITS
+    assert q(P, 4, 63, 4, 0, P, P, P, None) == wq.WQ_ERR_SHAPE
+    assert q(P, 0, 64, 4, 0, P, P, P, None) == wq.WQ_ERR_SHAPE
+    assert q(P, 4, 64, 4, 48, P, P, P, None) == wq.WQ_ERR_GROUP
+    assert q(P, 4, 64, 4, 16, P, P, P, None) == wq.WQ_ERR_GROUP
+    assert q(P + 8, 4, 64, 4, 32, P, P, P, None) == wq.WQ_ERR_ALIGN
+    g = L.wq_gemm
+    assert g(P, 1, 4, 64, P, P, P, 4, 32, None, None) == wq.WQ_ERR_NULL
+    assert g(P, 0, 4, 64, P, P, P, 4, 32, P, None) == wq.WQ_ERR_SHAPE
+    assert g(P, 1, 4, 64, P, P, P, 7, 32, P, None) == wq.WQ_ERR_BITS
+    assert g(P, 1, 4, 64, P, P, P, 4, 96, P, None) == wq.WQ_ERR_GROUP
+    assert g(P, 1, 4, 64, P, P, P + 4, 4, 32, P, None) == wq.WQ_ERR_ALIGN

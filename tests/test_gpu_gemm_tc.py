@@ -1,0 +1,83 @@
+"""Tensor-core GEMM (M > 16) vs the oracle: y within the stated tolerance."""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import wq_inputs
+from gpu_util import assert_y_close, cached_weight, oracle_quantize, to_dev_f16, wq
+
+pytestmark = pytest.mark.gpu
+
+BITS = (2, 3, 4, 8)
+
+
+def _run(Wh, x, bits, group):
+    N, K = Wh.shape
+    m = wq()
+    codes, s, z = m.wq_quantize_rtn(to_dev_f16(Wh), bits, group)
+    y = m.wq_gemm(x.cuda(), codes, s, z, bits, group, N, K)
+    torch.cuda.synchronize()
+    assert m.wq_last_device_error() == m.WQ_OK
+    oc, os_, oz = oracle_quantize(Wh, bits, group)
+    y_ref, bound = oracle.gemm(wq_inputs.bf16_bits(x), oc, os_, oz, N, K, bits, group)
+    return y.float().cpu().numpy(), y_ref, bound
+
+
+@pytest.mark.parametrize("bits", BITS)
+@pytest.mark.parametrize("M,N,K,group", [
+    (17, 256, 128, 128), (64, 300, 384, 32), (256, 256, 256, 0), (257, 200, 640, 128),
+    (520, 513, 384, 64)])
+def test_tc_small(bits, M, N, K, group):
+    Wh = wq_inputs.weight_f16(8, bits, N, K)
+    x = wq_inputs.activations_bf16(8, M, M, K)
+    y, yr, b = _run(Wh, x, bits, group)
+    assert_y_close(y, yr, b, f"bits={bits} M={M} N={N} K={K} g={group}")
+
+
+def test_tc_k_not_multiple_of_128_uses_gemv_chunks():
+    N, K, M, bits, group = 70, 4160, 40, 4, 32
+    Wh = wq_inputs.weight_f16(9, 0, N, K)
+    x = wq_inputs.activations_bf16(9, 1, M, K)
+    y, yr, b = _run(Wh, x, bits, group)
+    assert_y_close(y, yr, b, "K=4160 M=40")
+
+
+@pytest.mark.parametrize("bits", BITS)
+def test_tc_one_hot_exact(bits):
+    N, K, M, group = 256, 256, 32, 128
+    Wh = wq_inputs.weight_f16(10, bits, N, K)
+    m = wq()
+    codes, s, z = m.wq_quantize_rtn(to_dev_f16(Wh), bits, group)
+    oc, os_, oz = oracle_quantize(Wh, bits, group)
+    wq_ref = oracle.dequant(oracle.unpack(oc, K, bits), os_, oz, group)
+    x = torch.zeros(M, K, dtype=torch.bfloat16)
+    ks = [(7 * i) % K for i in range(M)]
+    for i, k in enumerate(ks):
+        x[i, k] = 1.0
+    y = m.wq_gemm(x.cuda(), codes, s, z, bits, group, N, K).cpu()
+    for i, k in enumerate(ks):
+        assert torch.equal(y[i], torch.from_numpy(wq_ref[:, k]).to(torch.bfloat16)), (i, k)
+
+
+@pytest.mark.parametrize("cfg,linear,M", [
+    ("llama13b_prefill_4b_g128", 0, 2048), ("llama13b_prefill_4b_g128", 1, 2048),
+    ("llama7b_stack32_4b_g128", 0, 64), ("llama7b_stack32_4b_g128", 6, 64)])
+def test_tc_full_size_sampled(cfg, linear, M):
+    w = wq_inputs.WORKLOADS[cfg]
+    name, N, K = w["linears"][linear]
+    bits, group = w["bits"], w["group"]
+    Wh = cached_weight(0, linear, N, K, w["dist"])
+    x = wq_inputs.activations_bf16(0, 200 + linear, M, K)
+    m = wq()
+    codes, s, z = m.wq_quantize_rtn(to_dev_f16(Wh), bits, group)
+    y = m.wq_gemm(x.cuda(), codes, s, z, bits, group, N, K).float().cpu().numpy()
+    assert m.wq_last_device_error() == m.WQ_OK
+    cols = np.unique(np.concatenate([[0, N - 1], np.random.default_rng(8).integers(0, N, 62)]))
+    rows = np.unique(np.concatenate([[0, M - 1], np.random.default_rng(9).integers(0, M, 30)]))
+    oc, os_, oz = oracle_quantize(Wh[cols], bits, group)
+    xs = x[torch.from_numpy(rows)]
+    y_ref, bound = oracle.gemm(wq_inputs.bf16_bits(xs), oc, os_, oz, len(cols), K, bits, group)
+    assert_y_close(y[np.ix_(rows, cols)], y_ref, bound, f"{cfg}/{name} M={M}")

@@ -1,0 +1,103 @@
+"""Decode GEMV (M <= 16) vs the oracle: y within the stated tolerance."""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import wq_inputs
+from gpu_util import assert_y_close, cached_weight, oracle_quantize, to_dev_f16, wq
+
+pytestmark = pytest.mark.gpu
+
+BITS = (2, 3, 4, 8)
+
+
+def _run(Wh, x, bits, group):
+    """Quantise on the GPU, multiply on the GPU; oracle from the same host bytes."""
+    N, K = Wh.shape
+    m = wq()
+    codes, s, z = m.wq_quantize_rtn(to_dev_f16(Wh), bits, group)
+    y = m.wq_gemm(x.cuda(), codes, s, z, bits, group, N, K)
+    torch.cuda.synchronize()
+    oc, os_, oz = oracle_quantize(Wh, bits, group)
+    y_ref, bound = oracle.gemm(wq_inputs.bf16_bits(x), oc, os_, oz, N, K, bits, group)
+    return y.float().cpu().numpy(), y_ref, bound
+
+
+@pytest.mark.parametrize("bits", BITS)
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 5, 8, 13, 16])
+def test_gemv_small(bits, M):
+    N, K, group = 70, 640, 128          # ragged N (3 CTAs), 20 blocks over 8 warps
+    Wh = wq_inputs.weight_f16(4, bits, N, K)
+    x = wq_inputs.activations_bf16(4, M, M, K)
+    y, yr, b = _run(Wh, x, bits, group)
+    assert_y_close(y, yr, b, f"bits={bits} M={M}")
+
+
+@pytest.mark.parametrize("bits", BITS)
+@pytest.mark.parametrize("group,K", [(32, 96), (64, 192), (0, 32), (0, 4160), (96, 288)])
+def test_gemv_groups_and_edges(bits, group, K):
+    N = 33
+    Wh = wq_inputs.weight_f16(5, bits, N, K, dist="t4")
+    for M in (1, 7):
+        x = wq_inputs.activations_bf16(5, M, M, K)
+        y, yr, b = _run(Wh, x, bits, group)
+        assert_y_close(y, yr, b, f"bits={bits} group={group} K={K} M={M}")
+
+
+@pytest.mark.parametrize("bits", BITS)
+def test_gemv_one_hot_exact(bits):
+    """A one-hot x selects one column of W': y must equal bf16(w') exactly."""
+    N, K, group = 64, 256, 64
+    Wh = wq_inputs.weight_f16(6, bits, N, K)
+    m = wq()
+    codes, s, z = m.wq_quantize_rtn(to_dev_f16(Wh), bits, group)
+    oc, os_, oz = oracle_quantize(Wh, bits, group)
+    wq_ref = oracle.dequant(oracle.unpack(oc, K, bits), os_, oz, group)
+    for k in (0, 5, 31, 32, 100, 255):
+        x = torch.zeros(3, K, dtype=torch.bfloat16)
+        x[0, k] = 1.0
+        x[2, k] = -2.0
+        y = m.wq_gemm(x.cuda(), codes, s, z, bits, group, N, K).cpu()
+        ref = torch.from_numpy(wq_ref[:, k]).to(torch.bfloat16)
+        assert torch.equal(y[0], ref)
+        assert torch.equal(y[1], torch.zeros(N, dtype=torch.bfloat16))
+        assert torch.equal(y[2], (-2.0 * torch.from_numpy(wq_ref[:, k])).to(torch.bfloat16))
+
+
+def test_gemv_zero_x_and_no_overwrite_beyond_y():
+    N, K, bits, group = 40, 128, 4, 32
+    Wh = wq_inputs.weight_f16(7, 0, N, K)
+    m = wq()
+    codes, s, z = m.wq_quantize_rtn(to_dev_f16(Wh), bits, group)
+    x = torch.zeros(2, K, dtype=torch.bfloat16, device="cuda")
+    buf = torch.full((2 * N + 64,), 7.0, dtype=torch.bfloat16, device="cuda")
+    y = buf[32:32 + 2 * N].view(2, N)
+    m.wq_gemm(x, codes, s, z, bits, group, N, K, y=y)
+    torch.cuda.synchronize()
+    assert torch.all(y == 0)
+    assert torch.all(buf[:32] == 7.0) and torch.all(buf[32 + 2 * N:] == 7.0)
+
+
+@pytest.mark.parametrize("cfg,linear,M", [
+    ("linear4096_4b_g128", 0, 1),
+    ("llama7b_layer_3b_g128", 0, 1), ("llama7b_layer_3b_g128", 1, 4),
+    ("llama7b_layer_3b_g128", 2, 16), ("llama7b_layer_3b_g128", 3, 1),
+    ("opt175b_fc_2b_rowwise", 0, 1), ("opt175b_fc_2b_rowwise", 1, 1),
+    ("opt175b_fc_8b_rowwise", 0, 1), ("opt175b_fc_8b_rowwise", 1, 1),
+    ("llama7b_stack32_4b_g128", 6, 16)])
+def test_gemv_full_size_sampled(cfg, linear, M):
+    w = wq_inputs.WORKLOADS[cfg]
+    name, N, K = w["linears"][linear]
+    bits, group = w["bits"], w["group"]
+    Wh = cached_weight(0, linear, N, K, w["dist"])
+    x = wq_inputs.activations_bf16(0, 100 + linear, M, K)
+    m = wq()
+    codes, s, z = m.wq_quantize_rtn(to_dev_f16(Wh), bits, group)
+    y = m.wq_gemm(x.cuda(), codes, s, z, bits, group, N, K).float().cpu().numpy()
+    cols = np.unique(np.concatenate([[0, N - 1], np.random.default_rng(7).integers(0, N, 126)]))
+    oc, os_, oz = oracle_quantize(Wh[cols], bits, group)
+    y_ref, bound = oracle.gemm(wq_inputs.bf16_bits(x), oc, os_, oz, len(cols), K, bits, group)
+    assert_y_close(y[:, cols], y_ref, bound, f"{cfg}/{name} M={M}")
