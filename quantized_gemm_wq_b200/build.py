@@ -61,7 +61,8 @@ def build(force: bool = False, verbose: bool = False, extra=()) -> str:
             sys.stderr.write(err)
     objs = [o for o, _ in results]
     tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [NVCC, *ARCH, "-shared", "-cudart", "static", "-Xcompiler", "-fPIC", *objs, "-o", tmp]
+    cmd = [NVCC, *ARCH, "-shared", "-cudart", "static", "-Xcompiler", "-fPIC",
+           "-Xlinker", "--no-undefined", *objs, "-o", tmp, "-ldl", "-lpthread", "-lrt"]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")

@@ -438,50 +438,16 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
 }
 
 // ------------------------------------------------------------------ host
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
-      return static_cast<EncodeTiledFn>(nullptr);
-    return reinterpret_cast<EncodeTiledFn>(p);
-  }();
-  return fn;
-}
-
 template <int BITS>
 cudaError_t launch_bits(const __nv_bfloat16* x, int64_t M, int64_t N, int64_t K,
                         const uint32_t* codes, const __half* scales, const __half* zeros,
                         int64_t g, __nv_bfloat16* y, cudaStream_t st) {
-  EncodeTiledFn enc = encode_fn();
-  if (!enc) return cudaErrorNotSupported;
-  CUtensorMap tx, tc;
-  {
-    const cuuint64_t dims[2] = {cuuint64_t(K), cuuint64_t(M)};
-    const cuuint64_t strides[1] = {cuuint64_t(K) * 2};
-    const cuuint32_t box[2] = {BK, BM};
-    const cuuint32_t es[2] = {1, 1};
-    if (enc(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<__nv_bfloat16*>(x), dims, strides,
-            box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return cudaErrorInvalidValue;
-  }
-  {
-    const cuuint64_t dims[2] = {cuuint64_t(K * BITS / 32), cuuint64_t(N)};
-    const cuuint64_t strides[1] = {cuuint64_t(K * BITS / 8)};
-    const cuuint32_t box[2] = {CK * BITS / 32, BN};
-    const cuuint32_t es[2] = {1, 1};
-    if (enc(&tc, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(codes), dims, strides,
-            box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return cudaErrorInvalidValue;
-  }
+  alignas(64) CUtensorMap tx, tc;
+  if (!make_tensor_map_2d(&tx, TmaType::kBF16, x, uint64_t(K), uint64_t(M), uint64_t(K) * 2, BK, BM,
+                          true) ||
+      !make_tensor_map_2d(&tc, TmaType::kU32, codes, uint64_t(K * BITS / 32), uint64_t(N),
+                          uint64_t(K * BITS / 8), CK * BITS / 32, BN, false))
+    return cudaErrorInvalidValue;
   constexpr uint32_t smem = TcCfg<BITS>::kSmem;
   static bool attr_set[64] = {};
   int dev = 0;
@@ -516,7 +482,7 @@ cudaError_t launch_gemm_tc(const __nv_bfloat16* x, int64_t M, int64_t N, int64_t
   }
 }
 
-bool read_and_clear_timeout_flag(cudaError_t* err) {
+bool gemm_tc_read_and_clear_timeout(cudaError_t* err) {
   unsigned int v = 0;
   const unsigned int zero = 0;
   cudaError_t e = cudaDeviceSynchronize();

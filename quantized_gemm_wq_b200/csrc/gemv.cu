@@ -8,43 +8,123 @@
 // bound when memory bandwidth limits decoding).  At M <= 16 the work is a scan
 // of the packed codes: every code byte is read from HBM exactly once.
 //
-// Work split.  A CTA owns 32 consecutive output rows (one per lane) and splits
-// their K dimension across its 8 warps (split-K across warps): warp w takes
-// tiles of U consecutive 32-code blocks, interleaved over warps.  Per block a
-// lane loads the b packed words of its row with one vector load (b = 2, 4, 8;
-// three 32-bit loads for b = 3), unpacks the 32 codes in registers and
-// accumulates  s * sum_k x[m,k] (q_k - z)  in fp32 for every batch row m.
-// The 32 x values of a block are staged once per warp in shared memory and read
-// as broadcasts.  Partial sums of the 8 warps are added through shared memory
-// at the end and y is rounded once to bf16.
+// Work split.  Each warp owns R consecutive output rows over the whole K.  A
+// lane owns one 32-code unit (b packed words) of every row per step, so one
+// warp-wide load reads 32 consecutive units of a row: 256/384/512/1024 bytes
+// contiguous for b = 2/3/4/8 (fully coalesced).  Steps are unrolled so that
+// R x S loads per lane are in flight before the first is used.  Each lane
+// keeps fp32 partial sums for its rows; a shuffle reduction across the 32
+// lanes (split-K over lanes) finishes every row.
 //
-// Exactness of the dequantisation: q - z is formed exactly as
-// float(0x4B000000 | q) - (2^23 + z): both terms are exact in fp32 (integers
-// below 2^24), so w' = s (q - z) is exact before the product with x.
+// Unpacking.  A code q sitting at bit p of a 32-bit word becomes a float with
+// one AND-OR (lop3): bits (word & (mask << p)) | ((150 - p) << 23) are the
+// float 2^(23-p) + q exactly (exponent 23 - p, q in the mantissa).  Every code
+// is brought to a position p in [8, 23 - b] by one of three shared word views
+// (word << 8 or 12, word, word >> 10..16 / a funnel shift for the b = 3
+// straddles), so a code costs one lop3.
+//   One FADD with the compile-time constant 2^(23-p) then gives q exactly, and
+//   q - z is formed exactly (M = 1: the zero is applied once per unit as
+//   s * (sum x q - z sum x), with sum x shared by the R rows; M > 1: q - z per
+//   code, reused for every batch row).  The constant is never folded into the
+//   accumulator: its rounding error would scale with sum |x| rather than with
+//   sum |x w'|, and rows whose codes sit mostly at the zero (outlier-heavy
+//   per-row grids) would lose the accuracy contract.
+// All products x * q and x * (q - z) are exact in fp32 (8-bit x significand
+// times a code of at most 9 bits); y is rounded once to bf16.
 #include "wq_internal.cuh"
 
 namespace wq {
 namespace {
 
-constexpr int kWarps = 8;
+constexpr int kWarps = 4;
 constexpr int kThreads = 32 * kWarps;
 
-template <int MT>
-struct GemvCfg {
-  static constexpr int U = MT <= 4 ? 4 : 2;   // blocks per warp tile (loads in flight)
+
+// ---------------------------------------------------------------- unpack plan
+// For code i (0..31) of a unit: the word it starts in, the view of that word
+// (0: shifted left, 1: as is, 2: shifted right / funnel), and its bit position
+// p in that view.
+struct Slot {
+  int word, view, p;
 };
 
 template <int BITS>
-__device__ __forceinline__ void load_codes(const uint32_t* __restrict__ p, uint32_t (&w)[BITS]) {
+__host__ __device__ constexpr int left_shift() { return BITS == 4 ? 12 : 8; }
+template <int BITS>
+__host__ __device__ constexpr int right_shift() {
+  return BITS == 2 ? 10 : BITS == 3 ? 12 : BITS == 4 ? 12 : 16;
+}
+
+template <int BITS>
+__host__ __device__ constexpr Slot slot(int i) {
+  const int bit = BITS * i;
+  const int word = bit / 32, P = bit % 32;
+  constexpr int L = left_shift<BITS>(), Rs = right_shift<BITS>();
+  if (BITS == 8) {           // one code per byte: a view per byte position
+    if (P == 0) return {word, 0, 8};
+    if (P == 8) return {word, 1, 8};
+    if (P == 16) return {word, 3, 8};   // >> 8
+    return {word, 2, 8};                // >> 16
+  }
+  if (P + L + BITS <= 23 && P + L >= 8) return {word, 0, P + L};
+  if (P + BITS <= 23 && P >= 8) return {word, 1, P};
+  return {word, 2, P - Rs};
+}
+
+template <int BITS>
+struct Views {
+  uint32_t v[BITS][4];
+};
+
+template <int BITS>
+__device__ __forceinline__ void make_views(const uint32_t (&w)[BITS], Views<BITS>& vw) {
+  constexpr int L = left_shift<BITS>(), Rs = right_shift<BITS>();
+#pragma unroll
+  for (int a = 0; a < BITS; ++a) {
+    vw.v[a][0] = w[a] << L;
+    vw.v[a][1] = w[a];
+    if constexpr (BITS == 3) {
+      vw.v[a][2] = (a < 2) ? __funnelshift_r(w[a], w[a + 1 < 3 ? a + 1 : 2], Rs) : (w[a] >> Rs);
+    } else {
+      vw.v[a][2] = w[a] >> Rs;
+    }
+    vw.v[a][3] = w[a] >> 8;
+  }
+}
+
+// (a & mask) | c in one lop3, mask an immediate and c a register.
+template <uint32_t MASK>
+__device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t c) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "n"(MASK), "r"(c));
+  return d;
+}
+
+// The float 2^(23-p) + q for code i.
+template <int BITS, int I>
+__device__ __forceinline__ float code_float(const Views<BITS>& vw) {
+  constexpr Slot s = slot<BITS>(I);
+  constexpr uint32_t mask = ((1u << BITS) - 1u) << s.p;
+  constexpr uint32_t expo = uint32_t(150 - s.p) << 23;
+  return __uint_as_float(and_or<mask>(vw.v[s.word][s.view], expo));
+}
+template <int BITS, int I>
+__host__ __device__ constexpr float code_bias() {
+  return float(1u << (23 - slot<BITS>(I).p));
+}
+
+// ---------------------------------------------------------------- loads
+template <int BITS>
+__device__ __forceinline__ void load_unit(const uint32_t* __restrict__ p, uint32_t (&w)[BITS]) {
   if constexpr (BITS == 2) {
-    uint2 v = __ldg(reinterpret_cast<const uint2*>(p));
+    const uint2 v = __ldg(reinterpret_cast<const uint2*>(p));
     w[0] = v.x; w[1] = v.y;
   } else if constexpr (BITS == 4) {
-    uint4 v = __ldg(reinterpret_cast<const uint4*>(p));
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(p));
     w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
   } else if constexpr (BITS == 8) {
-    uint4 a = __ldg(reinterpret_cast<const uint4*>(p));
-    uint4 b = __ldg(reinterpret_cast<const uint4*>(p) + 1);
+    const uint4 a = __ldg(reinterpret_cast<const uint4*>(p));
+    const uint4 b = __ldg(reinterpret_cast<const uint4*>(p) + 1);
     w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
     w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
   } else {
@@ -52,127 +132,255 @@ __device__ __forceinline__ void load_codes(const uint32_t* __restrict__ p, uint3
   }
 }
 
-// Code i (0..31) of a 32-code block, per the packed layout.
-template <int BITS>
-__device__ __forceinline__ uint32_t code_at(const uint32_t (&w)[BITS], int i) {
-  if constexpr (BITS == 3) {
-    const int bit = 3 * i, a = bit >> 5, sh = bit & 31;
-    const uint32_t nxt = (a + 1 < 3) ? w[(a + 1) % 3] : 0u;
-    return __funnelshift_r(w[a], nxt, sh) & 7u;
-  } else {
-    constexpr int per = 32 / BITS;
-    return (w[i / per] >> (BITS * (i % per))) & ((1u << BITS) - 1u);
+// 32 bf16 of x (one unit's k-range) as fp32.
+__device__ __forceinline__ void load_x32(const __nv_bfloat16* __restrict__ p, float (&x)[32]) {
+  const uint4* q = reinterpret_cast<const uint4*>(p);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint4 u = __ldg(q + j);
+    const uint32_t r[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      x[8 * j + 2 * t] = __uint_as_float(r[t] << 16);
+      x[8 * j + 2 * t + 1] = __uint_as_float(r[t] & 0xFFFF0000u);
+    }
   }
 }
 
-template <int BITS, int MT>
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+template <int BITS, int I>
+struct Unroll {
+  // sum_i x_i * f_i over codes I..31 (f: 2^(23-p) + q), and sum_i x_i 2^(23-p_i)
+  __device__ __forceinline__ static void dot(const float (&x)[32], const Views<BITS>& vw, float& d0,
+                                             float& d1) {
+    d0 = fmaf(x[I], code_float<BITS, I>(vw) - code_bias<BITS, I>(), d0);
+    if constexpr (I + 1 < 32) {
+      d1 = fmaf(x[I + 1], code_float<BITS, I + 1>(vw) - code_bias<BITS, I + 1>(), d1);
+      Unroll<BITS, I + 2>::dot(x, vw, d0, d1);
+    }
+  }
+  __device__ __forceinline__ static void xsum(const float (&x)[32], float& s) {
+    s += x[I];
+    if constexpr (I + 1 < 32) Unroll<BITS, I + 1>::xsum(x, s);
+  }
+  // exact q - z for codes I..I+7 (c: per-row zero; q = f - 2^(23-p) exactly)
+  __device__ __forceinline__ static void qz8(const Views<BITS>& vw, float z, float (&out)[8]) {
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      out[t] = 0.0f;
+    }
+    Fill<0>::run(vw, z, out);
+  }
+  template <int T>
+  struct Fill {
+    __device__ __forceinline__ static void run(const Views<BITS>& vw, float z, float (&out)[8]) {
+      out[T] = (code_float<BITS, I + T>(vw) - code_bias<BITS, I + T>()) - z;
+      if constexpr (T + 1 < 8) Fill<T + 1>::run(vw, z, out);
+    }
+  };
+};
+template <int BITS>
+struct Unroll<BITS, 32> {
+  __device__ __forceinline__ static void dot(const float (&)[32], const Views<BITS>&, float&, float&) {}
+  __device__ __forceinline__ static void xsum(const float (&)[32], float&) {}
+};
+
+// ---------------------------------------------------------------- M = 1
+template <int BITS, int R>
+struct Step {
+  uint32_t w[R][BITS];
+  float s[R], z[R];
+};
+
+template <int BITS, int R>
+__device__ __forceinline__ void load_step(Step<BITS, R>& st, const uint32_t* __restrict__ codes,
+                                          const __half* __restrict__ scales,
+                                          const __half* __restrict__ zeros, int64_t row0,
+                                          int64_t N, int64_t KW, int64_t G, int64_t u, int64_t KU,
+                                          const FastDiv& upg) {
+  const uint32_t grp = upg.div(uint32_t(u < KU ? u : 0));
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const int64_t n = row0 + r;
+    if (u < KU && n < N) {
+      load_unit<BITS>(codes + n * KW + u * BITS, st.w[r]);
+      st.s[r] = __half2float(scales[n * G + grp]);
+      st.z[r] = __half2float(zeros[n * G + grp]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < BITS; ++i) st.w[r][i] = 0u;
+      st.s[r] = 0.0f;
+      st.z[r] = 0.0f;
+    }
+  }
+}
+
+template <int BITS, int R>
+__device__ __forceinline__ void compute_step(const Step<BITS, R>& st, const __nv_bfloat16* __restrict__ xu,
+                                             float (&acc)[R]) {
+  float xf[32];
+  load_x32(xu, xf);
+  float sx = 0.0f;
+  Unroll<BITS, 0>::xsum(xf, sx);
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    Views<BITS> vw;
+    make_views<BITS>(st.w[r], vw);
+    float d0 = 0.0f, d1 = 0.0f;
+    Unroll<BITS, 0>::dot(xf, vw, d0, d1);
+    acc[r] = fmaf(st.s[r], fmaf(-st.z[r], sx, d0 + d1), acc[r]);
+  }
+}
+
+template <int BITS, int R>
+__global__ void __launch_bounds__(kThreads, 4)
+gemv1_kernel(const __nv_bfloat16* __restrict__ x, int64_t N, int64_t K,
+             const uint32_t* __restrict__ codes, const __half* __restrict__ scales,
+             const __half* __restrict__ zeros, FastDiv units_per_group,
+             __nv_bfloat16* __restrict__ y) {
+  const int lane = threadIdx.x & 31;
+  const int64_t row0 = (int64_t(blockIdx.x) * kWarps + (threadIdx.x >> 5)) * R;
+  if (row0 >= N) return;
+  const int64_t KU = K / 32;                 // units per row
+  const int64_t KW = K * BITS / 32;          // words per row
+  const int64_t G = K / (int64_t(units_per_group.d) * 32);
+  float acc[R];
+#pragma unroll
+  for (int r = 0; r < R; ++r) acc[r] = 0.0f;
+
+  // Two register buffers: the next step's codes are in flight while the
+  // current step is unpacked.
+  Step<BITS, R> a, b;
+  int64_t u = lane;
+  load_step<BITS, R>(a, codes, scales, zeros, row0, N, KW, G, u, KU, units_per_group);
+  while (u < KU) {
+    load_step<BITS, R>(b, codes, scales, zeros, row0, N, KW, G, u + 32, KU, units_per_group);
+    compute_step<BITS, R>(a, x + u * 32, acc);
+    u += 32;
+    if (u >= KU) break;
+    load_step<BITS, R>(a, codes, scales, zeros, row0, N, KW, G, u + 32, KU, units_per_group);
+    compute_step<BITS, R>(b, x + u * 32, acc);
+    u += 32;
+  }
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const float v = warp_sum(acc[r]);
+    if (lane == r && row0 + r < N) y[row0 + r] = __float2bfloat16_rn(v);
+  }
+}
+
+// ---------------------------------------------------------------- 2 <= M <= 16
+template <int BITS, int MT, int R>
 __global__ void __launch_bounds__(kThreads)
-gemv_kernel(const __nv_bfloat16* __restrict__ x, int M, int64_t N, int64_t K,
-            const uint32_t* __restrict__ codes, const __half* __restrict__ scales,
-            const __half* __restrict__ zeros, int64_t g, FastDiv blocks_per_group,
-            __nv_bfloat16* __restrict__ y) {
-  constexpr int U = GemvCfg<MT>::U;
-  constexpr int kStage = kWarps * U * MT * 32;
-  constexpr int kRed = kWarps * MT * 32;
-  __shared__ __align__(16) float smem[kStage > kRed ? kStage : kRed];
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t n = int64_t(blockIdx.x) * 32 + lane;
-  const bool row_ok = n < N;
-  const int64_t KB = K / 32;
+gemvm_kernel(const __nv_bfloat16* __restrict__ x, int M, int64_t N, int64_t K,
+             const uint32_t* __restrict__ codes, const __half* __restrict__ scales,
+             const __half* __restrict__ zeros, FastDiv units_per_group,
+             __nv_bfloat16* __restrict__ y) {
+  const int lane = threadIdx.x & 31;
+  const int64_t row0 = (int64_t(blockIdx.x) * kWarps + (threadIdx.x >> 5)) * R;
+  if (row0 >= N) return;
+  const int64_t KU = K / 32;
   const int64_t KW = K * BITS / 32;
-  const int64_t G = K / g;
-  const uint32_t* crow = codes + (row_ok ? n : 0) * KW;
-  const __half* srow = scales + (row_ok ? n : 0) * G;
-  const __half* zrow = zeros + (row_ok ? n : 0) * G;
-  float* xs = smem + warp * (U * MT * 32);
-
-  float acc[MT];
+  const int64_t G = K / (int64_t(units_per_group.d) * 32);
+  float acc[R][MT];
 #pragma unroll
-  for (int m = 0; m < MT; ++m) acc[m] = 0.0f;
-
-  for (int64_t t0 = int64_t(warp) * U; t0 < KB; t0 += int64_t(kWarps) * U) {
-    uint32_t cw[U][BITS];
-    float sc[U], zb[U];
+  for (int r = 0; r < R; ++r)
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int64_t kb = t0 + u;
-      if (row_ok && kb < KB) {
-        load_codes<BITS>(crow + kb * BITS, cw[u]);
-        const uint32_t grp = blocks_per_group.div(uint32_t(kb));
-        sc[u] = __half2float(srow[grp]);
-        zb[u] = 8388608.0f + __half2float(zrow[grp]);
+    for (int m = 0; m < MT; ++m) acc[r][m] = 0.0f;
+
+  for (int64_t u = lane; u < KU; u += 32) {
+    const uint32_t grp = units_per_group.div(uint32_t(u));
+    Views<BITS> vw[R];
+    float sc[R], zz[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int64_t n = row0 + r;
+      uint32_t w[BITS];
+      if (n < N) {
+        load_unit<BITS>(codes + n * KW + u * BITS, w);
+        sc[r] = __half2float(scales[n * G + grp]);
+        zz[r] = __half2float(zeros[n * G + grp]);
       } else {
 #pragma unroll
-        for (int i = 0; i < BITS; ++i) cw[u][i] = 0u;
-        sc[u] = 0.0f;
-        zb[u] = 8388608.0f;
+        for (int i = 0; i < BITS; ++i) w[i] = 0u;
+        sc[r] = 0.0f;
+        zz[r] = 0.0f;
       }
+      make_views<BITS>(w, vw[r]);
     }
+    float d[R][MT];
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int64_t kb = t0 + u;
+    for (int r = 0; r < R; ++r)
 #pragma unroll
-      for (int m = 0; m < MT; ++m) {
-        float v = 0.0f;
-        if (m < M && kb < KB) v = __bfloat162float(x[int64_t(m) * K + kb * 32 + lane]);
-        xs[(u * MT + m) * 32 + lane] = v;
+      for (int m = 0; m < MT; ++m) d[r][m] = 0.0f;
+    // 4 chunks of 8 codes: q - z per row once, then every batch row
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      float qz[R][8];
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        if (c == 0) Unroll<BITS, 0>::qz8(vw[r], zz[r], qz[r]);
+        else if (c == 1) Unroll<BITS, 8>::qz8(vw[r], zz[r], qz[r]);
+        else if (c == 2) Unroll<BITS, 16>::qz8(vw[r], zz[r], qz[r]);
+        else Unroll<BITS, 24>::qz8(vw[r], zz[r], qz[r]);
       }
-    }
-    __syncwarp();
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      float qz[32];
-#pragma unroll
-      for (int i = 0; i < 32; ++i)
-        qz[i] = __int_as_float(0x4B000000 | int(code_at<BITS>(cw[u], i))) - zb[u];
 #pragma unroll
       for (int m = 0; m < MT; ++m) {
         if (m < M) {
-          const float4* xv = reinterpret_cast<const float4*>(xs + (u * MT + m) * 32);
-          float d0 = 0.0f, d1 = 0.0f;
+          const uint4 xv = __ldg(reinterpret_cast<const uint4*>(x + int64_t(m) * K + u * 32 + 8 * c));
+          const uint32_t xr[4] = {xv.x, xv.y, xv.z, xv.w};
+          float xf[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const float4 xx = xv[i];
-            d0 = fmaf(xx.x, qz[4 * i + 0], d0);
-            d1 = fmaf(xx.y, qz[4 * i + 1], d1);
-            d0 = fmaf(xx.z, qz[4 * i + 2], d0);
-            d1 = fmaf(xx.w, qz[4 * i + 3], d1);
+          for (int t = 0; t < 4; ++t) {
+            xf[2 * t] = __uint_as_float(xr[t] << 16);
+            xf[2 * t + 1] = __uint_as_float(xr[t] & 0xFFFF0000u);
           }
-          acc[m] = fmaf(sc[u], d0 + d1, acc[m]);
+#pragma unroll
+          for (int r = 0; r < R; ++r)
+#pragma unroll
+            for (int t = 0; t < 8; ++t) d[r][m] = fmaf(xf[t], qz[r][t], d[r][m]);
         }
       }
     }
-    __syncwarp();
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+      for (int m = 0; m < MT; ++m) acc[r][m] = fmaf(sc[r], d[r][m], acc[r][m]);
   }
-
-  __syncthreads();   // staging area is reused for the cross-warp reduction
 #pragma unroll
-  for (int m = 0; m < MT; ++m) smem[(warp * MT + m) * 32 + lane] = acc[m];
-  __syncthreads();
-  for (int idx = threadIdx.x; idx < MT * 32; idx += kThreads) {
-    const int m = idx >> 5, l = idx & 31;
-    const int64_t nn = int64_t(blockIdx.x) * 32 + l;
-    if (m < M && nn < N) {
-      float s = 0.0f;
+  for (int r = 0; r < R; ++r)
 #pragma unroll
-      for (int w = 0; w < kWarps; ++w) s += smem[(w * MT + m) * 32 + l];
-      y[int64_t(m) * N + nn] = __float2bfloat16_rn(s);
+    for (int m = 0; m < MT; ++m) {
+      const float v = warp_sum(acc[r][m]);
+      if (lane == 0 && m < M && row0 + r < N) y[int64_t(m) * N + row0 + r] = __float2bfloat16_rn(v);
     }
-  }
 }
 
 template <int BITS>
 cudaError_t launch_bits(const __nv_bfloat16* x, int M, int64_t N, int64_t K,
                         const uint32_t* codes, const __half* scales, const __half* zeros,
                         int64_t g, __nv_bfloat16* y, cudaStream_t st) {
-  const dim3 grid(unsigned((N + 31) / 32));
-  const FastDiv bpg(uint32_t(g / 32));
-  if (M <= 1) gemv_kernel<BITS, 1><<<grid, kThreads, 0, st>>>(x, M, N, K, codes, scales, zeros, g, bpg, y);
-  else if (M <= 2) gemv_kernel<BITS, 2><<<grid, kThreads, 0, st>>>(x, M, N, K, codes, scales, zeros, g, bpg, y);
-  else if (M <= 4) gemv_kernel<BITS, 4><<<grid, kThreads, 0, st>>>(x, M, N, K, codes, scales, zeros, g, bpg, y);
-  else if (M <= 8) gemv_kernel<BITS, 8><<<grid, kThreads, 0, st>>>(x, M, N, K, codes, scales, zeros, g, bpg, y);
-  else gemv_kernel<BITS, 16><<<grid, kThreads, 0, st>>>(x, M, N, K, codes, scales, zeros, g, bpg, y);
+  const FastDiv upg(uint32_t(g / 32));
+  auto grid_for = [&](int R) { return dim3(unsigned((N + int64_t(kWarps) * R - 1) / (int64_t(kWarps) * R))); };
+  if (M <= 1) {
+    if (gemv_m1_tma_supported(K, BITS))   // rows start on 16 bytes: TMA-staged codes
+      return launch_gemv_m1_tma(x, N, K, codes, scales, zeros, BITS, g, y, st);
+    constexpr int R = BITS == 8 ? 2 : 4;
+    gemv1_kernel<BITS, R><<<grid_for(R), kThreads, 0, st>>>(x, N, K, codes, scales, zeros, upg, y);
+  } else if (M <= 2) {
+    gemvm_kernel<BITS, 2, 4><<<grid_for(4), kThreads, 0, st>>>(x, M, N, K, codes, scales, zeros, upg, y);
+  } else if (M <= 4) {
+    gemvm_kernel<BITS, 4, 4><<<grid_for(4), kThreads, 0, st>>>(x, M, N, K, codes, scales, zeros, upg, y);
+  } else if (M <= 8) {
+    gemvm_kernel<BITS, 8, 2><<<grid_for(2), kThreads, 0, st>>>(x, M, N, K, codes, scales, zeros, upg, y);
+  } else {
+    gemvm_kernel<BITS, 16, 2><<<grid_for(2), kThreads, 0, st>>>(x, M, N, K, codes, scales, zeros, upg, y);
+  }
   return cudaGetLastError();
 }
 

@@ -124,10 +124,11 @@ wq_status wq_gemm(const void* x_bf16, int64_t M, int64_t N, int64_t K, const uin
 }
 
 wq_status wq_last_device_error(void) {
-  cudaError_t e = cudaSuccess;
-  const bool hit = wq::read_and_clear_timeout_flag(&e);
-  if (e != cudaSuccess) return WQ_ERR_CUDA;
-  return hit ? WQ_ERR_DEVICE_TIMEOUT : WQ_OK;
+  cudaError_t e1 = cudaSuccess, e2 = cudaSuccess;
+  const bool hit1 = wq::gemm_tc_read_and_clear_timeout(&e1);
+  const bool hit2 = wq::gemv_m1_tma_read_and_clear_timeout(&e2);
+  if (e1 != cudaSuccess || e2 != cudaSuccess) return WQ_ERR_CUDA;
+  return (hit1 || hit2) ? WQ_ERR_DEVICE_TIMEOUT : WQ_OK;
 }
 
 }  // extern "C"

@@ -19,9 +19,9 @@ inline int64_t effective_group(int64_t K, int64_t group) { return (group == 0) ?
 // multiplication, Granlund & Montgomery 1994): l = ceil(log2 d),
 // m = floor(2^32 (2^l - d) / d) + 1, n / d = (mulhi(n, m) + n) >> l.
 struct FastDiv {
-  uint32_t m = 1, l = 0;
+  uint32_t m = 1, l = 0, d = 1;
   FastDiv() = default;
-  explicit FastDiv(uint32_t d) {
+  explicit FastDiv(uint32_t d_) : d(d_) {
     l = 0;
     while ((uint64_t(1) << l) < d) ++l;
     m = uint32_t(((uint64_t(1) << 32) * ((uint64_t(1) << l) - d)) / d + 1);
@@ -39,6 +39,13 @@ cudaError_t launch_gemv(const __nv_bfloat16* x, int M, int64_t N, int64_t K,
                         const uint32_t* codes, const __half* scales, const __half* zeros,
                         int bits, int64_t g, __nv_bfloat16* y, cudaStream_t st);
 
+// M = 1 decode GEMV with TMA-staged codes; needs 16-byte aligned code rows.
+bool gemv_m1_tma_supported(int64_t K, int bits);
+cudaError_t launch_gemv_m1_tma(const __nv_bfloat16* x, int64_t N, int64_t K,
+                               const uint32_t* codes, const __half* scales, const __half* zeros,
+                               int bits, int64_t g, __nv_bfloat16* y, cudaStream_t st);
+bool gemv_m1_tma_read_and_clear_timeout(cudaError_t* err);
+
 // True when the tensor-core path can stage this K with TMA (K a multiple of 128).
 bool gemm_tc_supported(int64_t K, int bits);
 
@@ -46,8 +53,13 @@ cudaError_t launch_gemm_tc(const __nv_bfloat16* x, int64_t M, int64_t N, int64_t
                            const uint32_t* codes, const __half* scales, const __half* zeros,
                            int bits, int64_t g, __nv_bfloat16* y, cudaStream_t st);
 
-// Reads and clears the device-side "bounded wait expired" flag of the current
-// device (synchronises the device).  Returns true if it was set.
-bool read_and_clear_timeout_flag(cudaError_t* err);
+// Reads and clears the device-side "bounded wait expired" flags of the current
+// device (synchronises the device).  Returns true if one was set.
+bool gemm_tc_read_and_clear_timeout(cudaError_t* err);
+
+// TMA tensor maps (a CUtensorMap is 128 bytes, 64-byte aligned).
+enum class TmaType { kU32, kBF16 };
+bool make_tensor_map_2d(void* map, TmaType type, const void* base, uint64_t inner, uint64_t outer,
+                        uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, bool swizzle128);
 
 }  // namespace wq
