@@ -36,6 +36,18 @@ namespace wq {
 namespace {
 
 constexpr int kScaleS = 64;
+
+// Resident CTAs per SM the register budget is sized for.
+#ifndef WQ_GEMV_M1_MIN_CTAS
+#define WQ_GEMV_M1_MIN_CTAS 2
+#endif
+// Split-K heuristic: CTAs wanted in total, and K stages kept per CTA.
+#ifndef WQ_GEMV_M1_TARGET_CTAS
+#define WQ_GEMV_M1_TARGET_CTAS 444
+#endif
+#ifndef WQ_GEMV_M1_MIN_STAGES
+#define WQ_GEMV_M1_MIN_STAGES 4
+#endif
 constexpr uint64_t kWaitNs = 1000000000ull;
 
 __device__ unsigned int g_gemv_tma_timeout;
@@ -69,6 +81,26 @@ __device__ __forceinline__ float code_subnormal(const uint32_t (&w)[BITS]) {
   return __uint_as_float(v & mask);
 }
 
+#ifndef WQ_GEMV_PAIRS
+#define WQ_GEMV_PAIRS 0
+#endif
+
+__device__ __forceinline__ uint64_t pack_f2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ uint64_t ffma_f2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ float2 unpack_f2(uint64_t v) {
+  float lo, hi;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+  return make_float2(lo, hi);
+}
+
 // d[I % 4] += x'[I] * f_I for I = I0..31 (four independent chains).
 template <int BITS, int I>
 struct Dot {
@@ -76,6 +108,16 @@ struct Dot {
                                              float (&d)[4]) {
     d[I & 3] = fmaf(xp[I], code_subnormal<BITS, I>(w), d[I & 3]);
     if constexpr (I + 1 < 32) Dot<BITS, I + 1>::run(w, xp, d);
+  }
+};
+// Same with packed f32x2 FMAs over code pairs (2 chains of pairs).
+template <int BITS, int J>
+struct Dot2 {
+  __device__ __forceinline__ static void run(const uint32_t (&w)[BITS], const uint64_t (&xp2)[16],
+                                             uint64_t (&d)[2]) {
+    d[J & 1] = ffma_f2(xp2[J], pack_f2(code_subnormal<BITS, 2 * J>(w), code_subnormal<BITS, 2 * J + 1>(w)),
+                       d[J & 1]);
+    if constexpr (J + 1 < 16) Dot2<BITS, J + 1>::run(w, xp2, d);
   }
 };
 
@@ -129,203 +171,313 @@ __device__ __forceinline__ void lds_words(uint32_t a, uint32_t (&w)[BITS]) {
   }
 }
 
-template <int BITS, int D>
-struct M1Cfg {
-  static constexpr int COL_BYTES = 32 * 16 * BITS;        // one box: 32 rows x 4 units
-  static constexpr int XS_BYTES = 2 * 128 * 4;             // staged x', double-buffered
-  // per-warp region, kept a multiple of 128 bytes (TMA destination alignment)
-  static constexpr int WARP_BYTES = (D * COL_BYTES + XS_BYTES + D * 8 + 127) / 128 * 128;
-};
 template <int BITS>
-constexpr int ring_depth() { return BITS == 8 ? 3 : 4; }
+struct M1Cfg {
+  static constexpr int NW = 8;                       // consumer warps (4 units of a stage each)
+  static constexpr int D = BITS == 8 ? 3 : 4;        // ring stages
+  static constexpr int STAGE_WORDS = 32 * BITS;      // 32 units of one row
+  static constexpr int BOX_BYTES = 32 * 128;         // one TMA box: 32 rows x 128 bytes, swizzled
+  static constexpr int STAGE_BYTES = BITS * BOX_BYTES;
+  static constexpr int XS_BYTES = NW * 2 * 128 * 4;  // per warp: staged x', double-buffered
+  static constexpr int SMEM = D * STAGE_BYTES + XS_BYTES + 2 * D * 8 + 1024;
+};
 
-template <int BITS, int W, int D>
-__global__ void __launch_bounds__(32 * W)
+// Shared-memory byte offset of word wi (0 .. 32*BITS-1) of row r in a stage:
+// the stage holds BITS boxes of 32 words per row; inside a box, rows are 128
+// bytes apart and the 16-byte chunk index is XOR-ed with r % 8 (128B swizzle).
+__device__ __forceinline__ uint32_t swz_word(int r, int wi) {
+  const int box = wi >> 5, c = (wi >> 2) & 7, e = wi & 3;
+  return uint32_t(box * 4096 + r * 128 + ((c ^ (r & 7)) << 4) + (e << 2));
+}
+
+// Shared-memory offsets of the pieces of unit u of row r in a stage: one
+// vector per 16-byte chunk (b = 2, 4, 8: 1, 1, 2 pieces) or one per word
+// (b = 3: 3 pieces).  They do not depend on the stage, so each lane computes
+// them once.
+template <int BITS>
+constexpr int unit_pieces() { return BITS == 3 ? 3 : (BITS == 8 ? 2 : 1); }
+
+template <int BITS>
+__device__ __forceinline__ void unit_offsets(int r, int u, uint32_t (&o)[unit_pieces<BITS>()]) {
+  if constexpr (BITS == 3) {
+#pragma unroll
+    for (int j = 0; j < 3; ++j) o[j] = swz_word(r, 3 * u + j);
+  } else if constexpr (BITS == 8) {
+    o[0] = swz_word(r, 8 * u);
+    o[1] = swz_word(r, 8 * u + 4);
+  } else {
+    o[0] = swz_word(r, BITS * u);
+  }
+}
+
+template <int BITS>
+__device__ __forceinline__ void load_unit_at(uint32_t stage, const uint32_t (&o)[unit_pieces<BITS>()],
+                                             uint32_t (&w)[BITS]) {
+  if constexpr (BITS == 4) {
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]) : "r"(stage + o[0]));
+  } else if constexpr (BITS == 2) {
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(w[0]), "=r"(w[1]) : "r"(stage + o[0]));
+  } else if constexpr (BITS == 8) {
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]) : "r"(stage + o[0]));
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(w[4]), "=r"(w[5]), "=r"(w[6]), "=r"(w[7]) : "r"(stage + o[1]));
+  } else {
+#pragma unroll
+    for (int j = 0; j < 3; ++j)
+      asm volatile("ld.shared.u32 %0, [%1];" : "=r"(w[j]) : "r"(stage + o[j]));
+  }
+}
+
+// One CTA: 32 output rows over the whole K.  Warp NW is the producer (one lane
+// issues the TMA copy of each 32-row x 32-unit box into a ring of D stages);
+// warps 0..NW-1 consume: warp w takes units 4w..4w+3 of every box, lane l
+// rows lr, lr+8, lr+16, lr+24 (lr = l % 8) of unit 4w + l / 8.  A stage is
+// released when every consumer warp has arrived on its "empty" barrier.
+template <int BITS>
+__global__ void __launch_bounds__(32 * (M1Cfg<BITS>::NW + 1), WQ_GEMV_M1_MIN_CTAS)
 gemv_m1_tma_kernel(const __grid_constant__ CUtensorMap tm_codes, const __nv_bfloat16* __restrict__ x,
                    int64_t N, int64_t K, const __half* __restrict__ scales,
                    const __half* __restrict__ zeros, FastDiv units_per_group,
                    __nv_bfloat16* __restrict__ y) {
-  using Cfg = M1Cfg<BITS, D>;
-  extern __shared__ __align__(128) uint8_t smem[];
-  __shared__ float red[W][32];
+  using Cfg = M1Cfg<BITS>;
+  constexpr int NW = Cfg::NW, D = Cfg::D;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  __shared__ float red[NW][32];
+  // the swizzle pattern repeats every 1024 bytes: align the ring to it
+  uint8_t* smem = smem_raw + ((1024 - (saddr(smem_raw) & 1023)) & 1023);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int lr = lane & 7, kq = lane >> 3;
-  uint8_t* wbase = smem + warp * Cfg::WARP_BYTES;
-  const uint32_t ring = saddr(wbase);
-  float* xs = reinterpret_cast<float*>(wbase + D * Cfg::COL_BYTES);
-  const uint32_t bar0 = saddr(wbase + D * Cfg::COL_BYTES + Cfg::XS_BYTES);
+  const uint32_t ring = saddr(smem);
+  const uint32_t full0 = saddr(smem + D * Cfg::STAGE_BYTES + Cfg::XS_BYTES);
+  const uint32_t empty0 = full0 + 8 * D;
 
   const int64_t row0 = int64_t(blockIdx.x) * 32;
   const int64_t KU = K / 32;
-  const int KC = int((KU + 3) / 4);
-  const int c0 = int(int64_t(KC) * warp / W), c1 = int(int64_t(KC) * (warp + 1) / W);
+  const int TT = int((KU + 31) / 32);                // stages along the whole K
+  // split-K over the CTAs of a cluster (gridDim.y = cluster size): this CTA
+  // takes stages [tb, te) and the partial sums meet in cluster rank 0
+  const int ks = int(gridDim.y), kr = int(blockIdx.y);
+  const int tb = int(int64_t(TT) * kr / ks), te = int(int64_t(TT) * (kr + 1) / ks);
+  const int T = te - tb;
   const int64_t G = K / (int64_t(units_per_group.d) * 32);
 
-  // x scale of code position `lane` (the position this lane stages).
-  const float xscale = __uint_as_float(uint32_t(127 + kScaleS - code_p<BITS>(lane)) << 23);
-
-  if (lane == 0) {
-    for (int s = 0; s < D; ++s)
-      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar0 + 8 * s));
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < D; ++s) {
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(full0 + 8 * s));
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(empty0 + 8 * s), "r"(NW));
+    }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  __syncwarp();
-  auto issue = [&](int c) {   // lane 0
-    if (c < c1) {
-      const int s = (c - c0) % D;
-      asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar0 + 8 * s),
-                   "r"(uint32_t(Cfg::COL_BYTES))
-                   : "memory");
-      asm volatile(
-          "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-          " [%0], [%1, {%3, %4}], [%2];" ::"r"(ring + s * Cfg::COL_BYTES),
-          "l"(&tm_codes), "r"(bar0 + 8 * s), "r"(c * 4 * BITS), "r"(int(row0))
-          : "memory");
-    }
-  };
-  // x of column c, position `lane` of its 4 units.
-  auto load_x = [&](int c, float (&xv)[4]) {
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int64_t k = (int64_t(c) * 4 + u) * 32 + lane;
-      xv[u] = (c < c1 && k < K) ? __bfloat162float(x[k]) : 0.0f;
-    }
-  };
-  // stage x' of a column and return sum x of this lane's unit kq.
-  auto stage_x = [&](int c, const float (&xv)[4]) {
-    float* dst = xs + ((c - c0) & 1) * 128;
-#pragma unroll
-    for (int u = 0; u < 4; ++u) dst[u * 32 + lane] = xv[u] * xscale;
-    const bool h16 = lane & 16, h8 = lane & 8;
-    float a = (h16 ? xv[2] : xv[0]) + __shfl_xor_sync(0xffffffffu, h16 ? xv[0] : xv[2], 16);
-    float b = (h16 ? xv[3] : xv[1]) + __shfl_xor_sync(0xffffffffu, h16 ? xv[1] : xv[3], 16);
-    float e = (h8 ? b : a) + __shfl_xor_sync(0xffffffffu, h8 ? a : b, 8);
-    e += __shfl_xor_sync(0xffffffffu, e, 4);
-    e += __shfl_xor_sync(0xffffffffu, e, 2);
-    e += __shfl_xor_sync(0xffffffffu, e, 1);
-    return e;
-  };
-  auto load_sz = [&](int c, float (&sc)[4], float (&zz)[4]) {
-    const int64_t ug = int64_t(c) * 4 + kq;
-    const uint32_t grp = units_per_group.div(uint32_t(ug < KU ? ug : 0));
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int64_t n = row0 + lr + 8 * i;
-      const bool ok = c < c1 && ug < KU && n < N;
-      sc[i] = ok ? __half2float(scales[n * G + grp]) : 0.0f;
-      zz[i] = ok ? __half2float(zeros[n * G + grp]) : 0.0f;
-    }
-  };
+  __syncthreads();
 
-  if (lane == 0)
-    for (int c = c0; c < c0 + D; ++c) issue(c);
-  float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-  float xv[4], sc[4], zz[4];
-  load_x(c0, xv);
-  float sx = stage_x(c0, xv);
-  load_sz(c0, sc, zz);
   bool ok = true;
-  int c = c0;
-  for (; c < c1; ++c) {
-    float xn[4], scn[4], zzn[4];
-    load_x(c + 1, xn);
-    load_sz(c + 1, scn, zzn);
-    const int s = (c - c0) % D;
-    ok = mbar_wait_bounded(bar0 + 8 * s, uint32_t(((c - c0) / D) & 1));
-    ok = __all_sync(0xffffffffu, ok);
-    if (!ok) break;
-    __syncwarp();                      // x' of column c is visible
-    float xp[32];
-    const float4* xq = reinterpret_cast<const float4*>(xs + ((c - c0) & 1) * 128 + kq * 32);
+  if (warp == NW) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0) {
+      for (int t = 0; t < T && ok; ++t) {
+        const int s = t % D;
+        if (t >= D) ok = mbar_wait_bounded(empty0 + 8 * s, uint32_t(((t / D) - 1) & 1));
+        if (!ok) break;
+        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(full0 + 8 * s),
+                     "r"(uint32_t(Cfg::STAGE_BYTES))
+                     : "memory");
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const float4 v = xq[j];
-      xp[4 * j] = v.x; xp[4 * j + 1] = v.y; xp[4 * j + 2] = v.z; xp[4 * j + 3] = v.w;
-    }
-    const uint32_t col = ring + uint32_t(s * Cfg::COL_BYTES);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      uint32_t w[BITS];
-      lds_words<BITS>(col + uint32_t((lr + 8 * i) * 16 * BITS + kq * 4 * BITS), w);
-      float d[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-      Dot<BITS, 0>::run(w, xp, d);
-      const float dot = (d[0] + d[1]) + (d[2] + d[3]);
-      acc[i] = fmaf(sc[i], fmaf(dot, 0x1p85f, -zz[i] * sx), acc[i]);
-    }
-    __syncwarp();                      // stage s and x' buffer (c - c0) & 1 are free again
-    if (lane == 0) issue(c + D);
-    sx = stage_x(c + 1, xn);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      sc[i] = scn[i];
-      zz[i] = zzn[i];
-    }
-  }
-  if (!ok) {                           // copies still in flight land before the CTA exits
-    if (lane == 0)
-      for (int k = c; k < c1 && k < c + D; ++k) {
-        const uint64_t t0 = now_ns();
-        while (!mbar_try(bar0 + 8 * ((k - c0) % D), uint32_t(((k - c0) / D) & 1)) &&
-               now_ns() - t0 < kWaitNs / 5) {
+        for (int b = 0; b < BITS; ++b)
+          asm volatile(
+              "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+              " [%0], [%1, {%3, %4}], [%2];" ::"r"(ring + s * Cfg::STAGE_BYTES + b * Cfg::BOX_BYTES),
+              "l"(&tm_codes), "r"(full0 + 8 * s), "r"((tb + t) * Cfg::STAGE_WORDS + 32 * b), "r"(int(row0))
+              : "memory");
+      }
+      if (!ok) {   // copies issued but not consumed must land before the CTA exits
+        for (int t = 0; t < T; ++t) {
+          const uint64_t t0 = now_ns();
+          while (!mbar_try(full0 + 8 * (t % D), uint32_t((t / D) & 1)) && now_ns() - t0 < kWaitNs / 5) {
+          }
         }
       }
-  }
+    }
+  } else {
+    // ---------------------------------------------------------------- consumers
+    const int lr = lane & 7, kq = lane >> 3;
+    float* xs = reinterpret_cast<float*>(smem + D * Cfg::STAGE_BYTES) + warp * 256;
+    const float xscale = __uint_as_float(uint32_t(127 + kScaleS - code_p<BITS>(lane)) << 23);
+    const bool rows_full = row0 + 32 <= N;
+    const __half* srow = scales + (row0 + lr) * G;
+    const __half* zrow = zeros + (row0 + lr) * G;
+    const int64_t G8 = 8 * G;
+    const int ub = 4 * warp;                           // this warp's first unit in a box
+
+    // x of box t, position `lane` of this warp's 4 units.
+    auto load_x = [&](int t, float (&xv)[4]) {
+      const int64_t u0 = int64_t(tb + t) * 32 + ub;
+      const __nv_bfloat16* xc = x + u0 * 32 + lane;
+      if (t < T && u0 + 4 <= KU) {
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    float v = acc[i];
-    v += __shfl_xor_sync(0xffffffffu, v, 8);
-    v += __shfl_xor_sync(0xffffffffu, v, 16);
-    if (kq == 0) red[warp][lr + 8 * i] = v;
+        for (int u = 0; u < 4; ++u) xv[u] = __bfloat162float(xc[32 * u]);
+      } else {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) xv[u] = (t < T && u0 + u < KU) ? __bfloat162float(xc[32 * u]) : 0.0f;
+      }
+    };
+    // stage x' of box t and return sum x of this lane's unit kq.
+    auto stage_x = [&](int t, const float (&xv)[4]) {
+      float* dst = xs + (t & 1) * 128;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) dst[u * 32 + lane] = xv[u] * xscale;
+      const bool h16 = lane & 16, h8 = lane & 8;
+      float a = (h16 ? xv[2] : xv[0]) + __shfl_xor_sync(0xffffffffu, h16 ? xv[0] : xv[2], 16);
+      float b = (h16 ? xv[3] : xv[1]) + __shfl_xor_sync(0xffffffffu, h16 ? xv[1] : xv[3], 16);
+      float e = (h8 ? b : a) + __shfl_xor_sync(0xffffffffu, h8 ? a : b, 8);
+      e += __shfl_xor_sync(0xffffffffu, e, 4);
+      e += __shfl_xor_sync(0xffffffffu, e, 2);
+      e += __shfl_xor_sync(0xffffffffu, e, 1);
+      return e;
+    };
+    auto load_sz = [&](int t, float (&sc)[4], float (&zz)[4]) {
+      const int64_t ug = int64_t(tb + t) * 32 + ub + kq;
+      const uint32_t grp = units_per_group.div(uint32_t(ug < KU ? ug : 0));
+      if (rows_full && t < T && ug < KU) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          sc[i] = __half2float(srow[i * G8 + grp]);
+          zz[i] = __half2float(zrow[i * G8 + grp]);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const bool in = t < T && ug < KU && row0 + lr + 8 * i < N;
+          sc[i] = in ? __half2float(srow[i * G8 + grp]) : 0.0f;
+          zz[i] = in ? __half2float(zrow[i * G8 + grp]) : 0.0f;
+        }
+      }
+    };
+
+    uint32_t uoff[4][unit_pieces<BITS>()];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) unit_offsets<BITS>(lr + 8 * i, ub + kq, uoff[i]);
+    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    float xv[4], sc[4], zz[4];
+    load_x(0, xv);
+    float sx = stage_x(0, xv);
+    load_sz(0, sc, zz);
+    for (int t = 0; t < T; ++t) {
+      float xn[4], scn[4], zzn[4];
+      load_x(t + 1, xn);
+      load_sz(t + 1, scn, zzn);
+      const int s = t % D;
+      ok = mbar_wait_bounded(full0 + 8 * s, uint32_t((t / D) & 1));
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      __syncwarp();                      // x' of box t is visible to every lane
+      const uint32_t stage = ring + uint32_t(s * Cfg::STAGE_BYTES);
+      float xp[32];
+      const float4* xq = reinterpret_cast<const float4*>(xs + (t & 1) * 128 + kq * 32);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float4 v = xq[j];
+        xp[4 * j] = v.x; xp[4 * j + 1] = v.y; xp[4 * j + 2] = v.z; xp[4 * j + 3] = v.w;
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        uint32_t w[BITS];
+        load_unit_at<BITS>(stage, uoff[i], w);
+        float d[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        Dot<BITS, 0>::run(w, xp, d);
+        const float dot = (d[0] + d[1]) + (d[2] + d[3]);
+        acc[i] = fmaf(sc[i], fmaf(dot, 0x1p85f, -zz[i] * sx), acc[i]);
+      }
+      __syncwarp();                      // this warp is done with stage s and x' buffer t & 1
+      if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(empty0 + 8 * s) : "memory");
+      sx = stage_x(t + 1, xn);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        sc[i] = scn[i];
+        zz[i] = zzn[i];
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float v = acc[i];
+      v += __shfl_xor_sync(0xffffffffu, v, 8);
+      v += __shfl_xor_sync(0xffffffffu, v, 16);
+      if (kq == 0) red[warp][lr + 8 * i] = v;
+    }
   }
   __syncthreads();
   if (threadIdx.x < 32) {
     float v = 0.0f;
 #pragma unroll
-    for (int w = 0; w < W; ++w) v += red[w][threadIdx.x];
+    for (int w = 0; w < NW; ++w) v += red[w][threadIdx.x];
+    red[0][threadIdx.x] = v;                        // this CTA's partial sums
+  }
+  if (ks > 1) {
+    // every CTA of the cluster has its partials in red[0]; rank 0 adds them
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+    if (kr == 0 && threadIdx.x < 32) {
+      float v = red[0][threadIdx.x];
+      const uint32_t mine = saddr(&red[0][threadIdx.x]);
+      for (int r = 1; r < ks; ++r) {
+        uint32_t peer;
+        float pv;
+        asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(peer) : "r"(mine), "r"(r));
+        asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(pv) : "r"(peer) : "memory");
+        v += pv;
+      }
+      red[0][threadIdx.x] = v;
+    }
+    // peers keep their shared memory until rank 0 has read it
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+  } else {
+    __syncthreads();
+  }
+  if (kr == 0 && threadIdx.x < 32) {
     const int64_t n = row0 + threadIdx.x;
-    if (n < N && ok) y[n] = __float2bfloat16_rn(v);
+    if (n < N) y[n] = __float2bfloat16_rn(red[0][threadIdx.x]);
   }
-}
-
-template <int BITS, int W>
-cudaError_t launch_w(const CUtensorMap& tm, const __nv_bfloat16* x, int64_t N, int64_t K,
-                     const __half* scales, const __half* zeros, const FastDiv& upg,
-                     __nv_bfloat16* y, cudaStream_t st) {
-  constexpr int D = ring_depth<BITS>();
-  constexpr int smem = W * M1Cfg<BITS, D>::WARP_BYTES;
-  static_assert(smem + W * 32 * 4 <= 232448, "shared memory");
-  static bool attr_set[64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    const cudaError_t e = cudaFuncSetAttribute(gemv_m1_tma_kernel<BITS, W, D>,
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
-  }
-  const dim3 grid(unsigned((N + 31) / 32));
-  gemv_m1_tma_kernel<BITS, W, D><<<grid, 32 * W, smem, st>>>(tm, x, N, K, scales, zeros, upg, y);
-  return cudaGetLastError();
 }
 
 template <int BITS>
 cudaError_t launch_bits(const __nv_bfloat16* x, int64_t N, int64_t K, const uint32_t* codes,
                         const __half* scales, const __half* zeros, int64_t g, __nv_bfloat16* y,
                         cudaStream_t st) {
+  using Cfg = M1Cfg<BITS>;
   alignas(64) CUtensorMap tm;
   if (!make_tensor_map_2d(&tm, TmaType::kU32, codes, uint64_t(K * BITS / 32), uint64_t(N),
-                          uint64_t(K * BITS / 8), 4 * BITS, 32, false))
+                          uint64_t(K * BITS / 8), 32, 32, true))
     return cudaErrorInvalidValue;
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    const cudaError_t e = cudaFuncSetAttribute(gemv_m1_tma_kernel<BITS>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  // Split K over a cluster of ks CTAs (at most 8) when the row tiles alone
+  // would leave SMs idle or run in a ragged second wave; every CTA keeps at
+  // least WQ_GEMV_M1_MIN_STAGES stages of K so its TMA ring still pipelines.
+  const int64_t tiles = (N + 31) / 32;
+  const int64_t stages = (K / 32 + 31) / 32;
+  int ks = int((WQ_GEMV_M1_TARGET_CTAS + tiles - 1) / tiles);
+  ks = ks < 1 ? 1 : (ks > 8 ? 8 : ks);
+  while (ks > 1 && stages / ks < WQ_GEMV_M1_MIN_STAGES) --ks;
   const FastDiv upg(uint32_t(g / 32));
-  // Warps per CTA: enough warps in total to cover every SM several times, but
-  // no more warps than box columns in a row.
-  const int64_t ctas = (N + 31) / 32;
-  const int64_t cols = (K / 32 + 3) / 4;
-  const int64_t want = (148 * 24 + ctas - 1) / ctas;
-  if (BITS != 8 && want >= 16 && cols >= 16)
-    return launch_w<BITS, (BITS == 8 ? 8 : 16)>(tm, x, N, K, scales, zeros, upg, y, st);
-  if (want >= 8 && cols >= 8) return launch_w<BITS, 8>(tm, x, N, K, scales, zeros, upg, y, st);
-  return launch_w<BITS, 4>(tm, x, N, K, scales, zeros, upg, y, st);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(unsigned(tiles), unsigned(ks), 1);
+  cfg.blockDim = dim3(32 * (Cfg::NW + 1), 1, 1);
+  cfg.dynamicSmemBytes = Cfg::SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = unsigned(ks);
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, gemv_m1_tma_kernel<BITS>, tm, x, N, K, scales, zeros, upg, y);
 }
 
 }  // namespace
