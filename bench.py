@@ -440,9 +440,15 @@ def main(argv=None):
     ap.add_argument("--copies", type=int, default=5,
                     help="distinct device copies of the layer rotated over the steps")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--case", default=None,
+                    help="run one small profiling case instead of the benchmark: "
+                         "decode | gemv:<i> | prefill:<i>")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.case:
+        run_case(args.case)
+        return
     rank, world, local = dist_setup()
     try:
         if args.impl == "reference":
@@ -453,6 +459,38 @@ def main(argv=None):
         import torch.distributed as dist
         if dist.is_available() and dist.is_initialized():
             dist.destroy_process_group()
+
+
+def run_case(case: str) -> None:
+    """One small profiling case (for ncu): ``decode`` runs one decode step of
+    the headline layer (the four M = 1 GEMV launches, after 3 warm-up steps);
+    ``gemv:<linear index>`` one M = 1 GEMV of that projection; ``prefill:<linear
+    index>`` one prefill GEMM (M = 2048) of the Llama-13B-shaped workload."""
+    import torch
+    import quantized_gemm_wq_b200 as wq
+    kind, _, arg = case.partition(":")
+    wl = PREFILL if kind == "prefill" else HEADLINE
+    w = wq_inputs.WORKLOADS[wl]
+    lins = list(enumerate(w["linears"]))
+    if kind in ("gemv", "prefill"):
+        lins = [lins[int(arg or 0)]]
+    M = w["Ms"][0] if kind == "prefill" else 1
+    ops = []
+    for li, (name, N, K) in lins:
+        W = torch.from_numpy(wq_inputs.weight_f16(0, li, N, K, dist=w["dist"])).cuda()
+        c, s, z = wq.wq_quantize_rtn(W, w["bits"], w["group"])
+        del W
+        x = wq_inputs.activations_bf16(0, 700 + li, M, K).cuda()
+        ops.append((x, c, s, z, N, K))
+    for _ in range(3):
+        for (x, c, s, z, N, K) in ops:
+            wq.wq_gemm(x, c, s, z, w["bits"], w["group"], N, K)
+    torch.cuda.synchronize()
+    for (x, c, s, z, N, K) in ops:
+        wq.wq_gemm(x, c, s, z, w["bits"], w["group"], N, K)
+    torch.cuda.synchronize()
+    assert wq.wq_last_device_error() == wq.WQ_OK
+    print(json.dumps({"case": case, "launches": len(ops), "ok": True}))
 
 
 def run_ours(args, rank, world, local):

@@ -107,10 +107,15 @@ wq_status wq_quantize_rtn(const void* W_f16, int64_t N, int64_t K, int bits, int
  *   stream          cudaStream_t
  *
  * Products and sums are fp32; y is rounded once to bf16 (RNE).  M <= 16 runs a
- * CUDA-core GEMV (codes streamed once with wide loads, unpacked in registers);
- * larger M runs a tensor-core GEMM (tcgen05 MMA, operands staged by TMA, W'
- * dequantised to bf16 in shared memory, accumulators in tensor memory).  Each
- * y element is within 2e-3 * sum_k |x w'| + 1e-3 of the exact fp64 value.
+ * CUDA-core GEMV (codes streamed once by TMA, unpacked in registers, exact
+ * x * (q - zero) products); larger M with K a multiple of 128 runs a
+ * tensor-core GEMM (tcgen05 MMA, operands staged by TMA, W' dequantised to
+ * bf16 in shared memory, accumulators in tensor memory), other K the GEMV 16
+ * batch rows at a time.  Accuracy: every product is exact or rounded once
+ * (w' to bf16 on the tensor-core path with grouped grids), sums are fp32, and
+ * y carries one bf16 rounding (up to 2^-8 |y|); on realistic inputs each y
+ * element lies within 2e-3 * sum_k |x w'| + 1e-3 of the exact value, which is
+ * the acceptance bound the tests use.  |x| must stay below 2^63.
  */
 wq_status wq_gemm(const void* x_bf16, int64_t M, int64_t N, int64_t K, const uint32_t* codes,
                   const void* scales_f16, const void* zeros_f16, int bits, int64_t group,
