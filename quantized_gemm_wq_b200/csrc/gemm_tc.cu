@@ -40,6 +40,13 @@ __device__ unsigned int g_timeout_flag;
 namespace {
 
 constexpr int BM = 256, BN = 256, BK = 64, CK = 128;
+
+#ifndef WQ_GEMM_MAX_SPLIT
+#define WQ_GEMM_MAX_SPLIT 4   // largest split-K cluster
+#endif
+#ifndef WQ_GEMM_MIN_STAGES
+#define WQ_GEMM_MIN_STAGES 8  // 128-wide code stages each split keeps at least
+#endif
 constexpr int kMmaM = 128, kMmaN = 256, kMmaK = 16;
 constexpr int kDqWarps = 8;
 constexpr int kThreads = 64 + 32 * kDqWarps;
@@ -170,6 +177,19 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
                : "memory");
 }
 
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// 16-byte load from the same shared-memory offset in cluster rank `rank`.
+__device__ __forceinline__ float4 ld_peer_f4(const void* p, int rank) {
+  uint32_t peer;
+  float4 v;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(peer) : "r"(smem_u32(p)), "r"(rank));
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(peer) : "memory");
+  return v;
+}
+
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
@@ -184,18 +204,27 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-// Code i (0..31) of a 32-code unit (layout of include/wq.h).
-template <int BITS>
-__device__ __forceinline__ uint32_t unit_code(const uint32_t (&w)[BITS], int i) {
-  if constexpr (BITS == 3) {
-    const int bit = 3 * i, a = bit >> 5, sh = bit & 31;
-    const uint32_t nxt = (a + 1 < 3) ? w[(a + 1) % 3] : 0u;
-    return __funnelshift_r(w[a], nxt, sh) & 7u;
-  } else {
-    constexpr int per = 32 / BITS;
-    return (w[i / per] >> (BITS * (i % per))) & ((1u << BITS) - 1u);
-  }
+constexpr float pow2f(int e) {
+  float r = 1.0f;
+  for (int i = 0; i < e; ++i) r *= 2.0f;
+  return r;
 }
+
+__device__ __forceinline__ uint32_t bf162_bits(float a, float b);
+
+// bf16 pairs (codes 2j, 2j+1 of a unit) of w' = fma(q 2^-30, A, B), j = J..15.
+template <int BITS, int J>
+struct DqPairs {
+  __device__ __forceinline__ static void run(const uint32_t (&w)[BITS], float A, float B,
+                                             uint32_t (&out)[16]) {
+    constexpr float F0 = pow2f(119 - code_p<BITS>(2 * J));
+    constexpr float F1 = pow2f(119 - code_p<BITS>(2 * J + 1));
+    const float a = fmaf(code_subnormal<BITS, 2 * J>(w) * F0, A, B);
+    const float b = fmaf(code_subnormal<BITS, 2 * J + 1>(w) * F1, A, B);
+    out[J] = bf162_bits(a, b);
+    if constexpr (J + 1 < 16) DqPairs<BITS, J + 1>::run(w, A, B, out);
+  }
+};
 
 template <int BITS>
 __device__ __forceinline__ void lds_unit(const uint8_t* p, uint32_t (&w)[BITS]) {
@@ -249,6 +278,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t n0 = int64_t(blockIdx.x) * BN, m0 = int64_t(blockIdx.y) * BM;
   const int KT = int((K + BK - 1) / BK);
+  // Split-K over the CTAs of a cluster (gridDim.z of them): this CTA takes the
+  // 128-wide code stages [cb, ce), i.e. K steps [kt0, kt1); the partial tiles
+  // are added in cluster rank 0 through distributed shared memory.
+  const int ks = int(gridDim.z), kr = int(blockIdx.z);
+  const int KC = (KT + 1) / 2;
+  const int kt0 = 2 * int(int64_t(KC) * kr / ks);
+  const int kt1 = min(KT, 2 * int(int64_t(KC) * (kr + 1) / ks));
   const bool rowwise = (g == K);
 
   if (threadIdx.x == 0) {
@@ -275,23 +311,25 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  bool ep_ok = false;                         // dequant warps: accumulators are final
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       int issued_a = 0, issued_c = 0;
       bool ok = true;
-      for (int kt = 0; kt < KT && ok; ++kt) {
-        if ((kt & 1) == 0) {                            // codes for K [kt*64, kt*64 + 128)
-          const int c = kt >> 1, cs = c % SC;
+      for (int kt = kt0; kt < kt1 && ok; ++kt) {
+        const int j = kt - kt0;                         // local step (ring phase)
+        if ((j & 1) == 0) {                             // codes for K [kt*64, kt*64 + 128)
+          const int c = j >> 1, cs = c % SC;
           if (c >= SC) ok = mbar_wait(&empty_c[cs], ((c / SC) - 1) & 1, abort);
           if (!ok) break;
           mbar_expect_tx(&full_c[cs], Cfg::kCBytes);
-          tma_load_2d(sC + cs * Cfg::kCBytes, &tm_c, &full_c[cs], c * (CK * BITS / 32), int(n0));
+          tma_load_2d(sC + cs * Cfg::kCBytes, &tm_c, &full_c[cs], (kt >> 1) * (CK * BITS / 32), int(n0));
           ++issued_c;
         }
-        const int s = kt % S;
-        if (kt >= S) ok = mbar_wait(&empty_ab[s], ((kt / S) - 1) & 1, abort);
+        const int s = j % S;
+        if (j >= S) ok = mbar_wait(&empty_ab[s], ((j / S) - 1) & 1, abort);
         if (!ok) break;
         mbar_expect_tx(&full_a[s], kABytes);
         tma_load_2d(sA + s * kABytes, &tm_x, &full_a[s], kt * BK, int(m0));
@@ -308,9 +346,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       bool ok = true;
-      for (int kt = 0; kt < KT && ok; ++kt) {
-        const int s = kt % S;
-        const uint32_t par = (kt / S) & 1;
+      for (int kt = kt0; kt < kt1 && ok; ++kt) {
+        const int s = (kt - kt0) % S;
+        const uint32_t par = ((kt - kt0) / S) & 1;
         ok = mbar_wait(&full_a[s], par, abort) && mbar_wait(&full_b[s], par, abort);
         if (!ok) break;
         tc_fence_after();
@@ -322,7 +360,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
 #pragma unroll
           for (int mt = 0; mt < BM / kMmaM; ++mt) {
             const uint64_t ad = sw128_desc(a0 + mt * (kMmaM * 128) + kk * kMmaK * 2);
-            umma(tmem + uint32_t(mt * kMmaN), ad, bd, (kt > 0 || kk > 0) ? 1u : 0u);
+            umma(tmem + uint32_t(mt * kMmaN), ad, bd, (kt > kt0 || kk > 0) ? 1u : 0u);
           }
         }
         umma_commit(&empty_ab[s]);
@@ -339,69 +377,125 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
       col_scale[c] = (n0 + c < N) ? __half2float(scales[(n0 + c) * G]) : 0.0f;
       asm volatile("bar.sync 1, %0;" ::"n"(32 * kDqWarps) : "memory");
     }
+    // Per thread: rows r0 = 32 dw + lane / 2 and r0 + 16 of the tile, unit cu of
+    // every 64-wide K step.  w' = s (q - z) = fma(q 2^-30, s 2^30, -s z): the
+    // code comes out of one AND as the subnormal float q 2^(p-149), one FMUL by
+    // 2^(119-p) (exact) gives q 2^-30, and the FMA is exact (s q and s z have at
+    // most 20 significant bits); the bf16 conversion is the only rounding.
+    // Scale and zero of the next step are loaded one step ahead.
+    const int r0 = 32 * dw + (lane >> 1);
+    auto load_ab = [&](int kt, float (&A)[2], float (&B)[2]) {
+      const int64_t k = int64_t(kt) * BK + 32 * cu;
+      const uint32_t grp = units_per_group.div(uint32_t(k >> 5));
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const int64_t n = n0 + r0 + 16 * i;
+        A[i] = 0.0f;
+        B[i] = 0.0f;
+        if (kt < kt1 && n < N && k < K) {
+          const float sc = rowwise ? 1.0f : __half2float(scales[n * G + grp]);
+          A[i] = sc * 0x1p30f;
+          B[i] = -sc * __half2float(zeros[n * G + grp]);
+        }
+      }
+    };
+    float A[2], B[2];
+    load_ab(kt0, A, B);
     bool ok = true;
-    for (int kt = 0; kt < KT && ok; ++kt) {
-      const int c = kt >> 1, cs = c % SC, s = kt % S;
+    for (int kt = kt0; kt < kt1 && ok; ++kt) {
+      const int j = kt - kt0;
+      const int c = j >> 1, cs = c % SC, s = j % S;
+      float An[2], Bn[2];
+      load_ab(kt + 1, An, Bn);
       ok = mbar_wait(&full_c[cs], (c / SC) & 1, abort);
-      if (ok && kt >= S) ok = mbar_wait(&empty_ab[s], ((kt / S) - 1) & 1, abort);
+      if (ok && j >= S) ok = mbar_wait(&empty_ab[s], ((j / S) - 1) & 1, abort);
       ok = __all_sync(0xffffffffu, ok);      // the warp leaves the loop together
       if (!ok) break;
       const uint8_t* ctile = sC + cs * Cfg::kCBytes;
       uint8_t* btile = sB + s * kBBytes;
-      const int64_t k = int64_t(kt) * BK + 32 * cu;
       const int ucode = (kt & 1) * 2 + cu;   // unit index within the 128-code stage
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
-        const int r = 32 * dw + (lane >> 1) + 16 * i;
-        const int64_t n = n0 + r;
-        float sc = 0.0f, zb = 8388608.0f;
-        if (n < N && k < K) {
-          const uint32_t grp = units_per_group.div(uint32_t(k >> 5));
-          sc = rowwise ? 1.0f : __half2float(scales[n * G + grp]);
-          zb = 8388608.0f + __half2float(zeros[n * G + grp]);
-        }
+        const int r = r0 + 16 * i;
         uint32_t w[BITS];
         lds_unit<BITS>(ctile + r * (CK * BITS / 8) + ucode * (4 * BITS), w);
+        uint32_t p[16];
+        DqPairs<BITS, 0>::run(w, A[i], B[i], p);
         uint8_t* brow = btile + r * 128;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          uint32_t p[4];
-#pragma unroll
-          for (int t = 0; t < 4; ++t) {
-            const int i0 = 8 * j + 2 * t;
-            const float a = (__int_as_float(0x4B000000 | int(unit_code<BITS>(w, i0))) - zb) * sc;
-            const float b = (__int_as_float(0x4B000000 | int(unit_code<BITS>(w, i0 + 1))) - zb) * sc;
-            p[t] = bf162_bits(a, b);
-          }
           const int chunk = (cu * 4 + j) ^ (r & 7);
-          *reinterpret_cast<uint4*>(brow + chunk * 16) = make_uint4(p[0], p[1], p[2], p[3]);
+          *reinterpret_cast<uint4*>(brow + chunk * 16) = make_uint4(p[4 * j], p[4 * j + 1], p[4 * j + 2], p[4 * j + 3]);
         }
       }
       fence_async_smem();
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(&full_b[s]);
-        if (kt & 1 || kt == KT - 1) mbar_arrive(&empty_c[cs]);
+        if ((j & 1) || kt == kt1 - 1) mbar_arrive(&empty_c[cs]);
+      }
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        A[i] = An[i];
+        B[i] = Bn[i];
       }
     }
-    // ------------------------------------------------------------ epilogue
     if (ok) ok = mbar_wait(tmem_full, 0, abort);
-    ok = __all_sync(0xffffffffu, ok);        // tcgen05.ld needs the whole warp
-    if (ok) {
+    ep_ok = __all_sync(0xffffffffu, ok);     // tcgen05.ld needs the whole warp
+  }
+
+  // ------------------------------------------------------------ epilogue
+  // Accumulator mt (rows 128 mt .. 128 mt + 127 of the tile) is written out by
+  // the 8 dequant warps: warp w reads TMEM lane quarter w % 4 and 128 of the 256
+  // columns.  With split-K, ranks > 0 first park their partial tile in their
+  // own (now idle) shared memory as [column / 4][row][4] floats, and rank 0
+  // adds them in through distributed shared memory.  Every thread takes part
+  // in the cluster barriers.
+  const bool dq = warp >= 2;
+  const int q = warp & 3;                    // TMEM lane quarter this warp may access
+  const int ch = (warp - 2) >> 2;            // column half
+  float4* part = reinterpret_cast<float4*>(sA);
+  const bool vec = (N % 8) == 0;
+  for (int mt = 0; mt < BM / kMmaM; ++mt) {
+    const int row = 32 * q + lane;           // row within accumulator mt
+    const uint32_t tbase = tmem + (uint32_t(32 * q) << 16) + uint32_t(mt * kMmaN);
+    if (ks > 1 && kr != 0 && dq && ep_ok) {
       tc_fence_after();
-      const int q = warp & 3;                  // TMEM lane quarter this warp may access
-      const int mt = dw >> 2;
-      const int64_t m = m0 + mt * kMmaM + 32 * q + lane;
-      const bool vec = (N % 8) == 0;
-      for (int cb = 0; cb < kMmaN / 32; ++cb) {
+      for (int cb = 0; cb < 4; ++cb) {
+        const int col0 = 128 * ch + 32 * cb;
         uint32_t r[32];
-        tmem_ld32(tmem + (uint32_t(32 * q) << 16) + uint32_t(mt * kMmaN + cb * 32), r);
+        tmem_ld32(tbase + uint32_t(col0), r);
+#pragma unroll
+        for (int v = 0; v < 8; ++v)
+          part[((col0 >> 2) + v) * 128 + row] =
+              make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                          __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
+      }
+    }
+    if (ks > 1) cluster_sync();
+    if (kr == 0 && dq && ep_ok) {
+      tc_fence_after();
+      const int64_t m = m0 + mt * kMmaM + row;
+      for (int cb = 0; cb < 4; ++cb) {
+        const int col0 = 128 * ch + 32 * cb;
+        uint32_t r[32];
+        tmem_ld32(tbase + uint32_t(col0), r);
+        for (int pr = 1; pr < ks; ++pr) {
+#pragma unroll
+          for (int v = 0; v < 8; ++v) {
+            const float4 pv = ld_peer_f4(&part[((col0 >> 2) + v) * 128 + row], pr);
+            r[4 * v] = __float_as_uint(__uint_as_float(r[4 * v]) + pv.x);
+            r[4 * v + 1] = __float_as_uint(__uint_as_float(r[4 * v + 1]) + pv.y);
+            r[4 * v + 2] = __float_as_uint(__uint_as_float(r[4 * v + 2]) + pv.z);
+            r[4 * v + 3] = __float_as_uint(__uint_as_float(r[4 * v + 3]) + pv.w);
+          }
+        }
         if (rowwise) {
 #pragma unroll
           for (int j = 0; j < 32; ++j)
-            r[j] = __float_as_uint(__uint_as_float(r[j]) * col_scale[cb * 32 + j]);
+            r[j] = __float_as_uint(__uint_as_float(r[j]) * col_scale[col0 + j]);
         }
-        const int64_t n = n0 + cb * 32;
+        const int64_t n = n0 + col0;
         if (m < M && n < N) {
           __nv_bfloat16* dst = y + m * N + n;
           if (vec && n + 32 <= N) {
@@ -422,6 +516,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         }
       }
     }
+    if (ks > 1) cluster_sync();              // peers keep their partials until read
   }
 
   // ------------------------------------------------------------ teardown
@@ -438,6 +533,39 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
 }
 
 // ------------------------------------------------------------------ host
+constexpr double kWaveStages = 5.0;    // prologue + epilogue of one wave, in code stages
+constexpr double kSplitStages = 3.0;   // partial-tile exchange per extra split
+
+// Clusters of c CTAs (one per SM, `smem` bytes each) resident at once; cached
+// per device and cluster size.  0 if the query fails.
+template <int BITS>
+int cluster_slots(int dev, int c, uint32_t smem) {
+  static int cache[64][4] = {};
+  int ci = 0;
+  while ((1 << ci) < c) ++ci;
+  if (dev < 0 || dev >= 64 || ci > 3) return 0;
+  if (cache[dev][ci] != 0) return cache[dev][ci] > 0 ? cache[dev][ci] : 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(1, 1, unsigned(c));
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = unsigned(c);
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, gemm_tc_kernel<BITS>, &cfg) != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    cache[dev][ci] = -1;
+    return 0;
+  }
+  cache[dev][ci] = n;
+  return n;
+}
+
 template <int BITS>
 cudaError_t launch_bits(const __nv_bfloat16* x, int64_t M, int64_t N, int64_t K,
                         const uint32_t* codes, const __half* scales, const __half* zeros,
@@ -458,10 +586,40 @@ cudaError_t launch_bits(const __nv_bfloat16* x, int64_t M, int64_t N, int64_t K,
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  const dim3 grid(unsigned((N + BN - 1) / BN), unsigned((M + BM - 1) / BM));
-  gemm_tc_kernel<BITS><<<grid, kThreads, smem, st>>>(tx, tc, scales, zeros, M, N, K, g,
-                                                      FastDiv(uint32_t(g / 32)), y);
-  return cudaGetLastError();
+  // Split K over a cluster when the output tiles alone fill the SMs badly.
+  // Cost model in units of one 128-wide code stage: every wave of clusters
+  // takes its share of K plus a fixed prologue/epilogue and a reduction cost
+  // per extra split; the cluster slots per wave come from the occupancy API
+  // (clusters of c CTAs of this size do not always pack the SMs fully).
+  const int64_t tiles = ((N + BN - 1) / BN) * ((M + BM - 1) / BM);
+  const int64_t kc = K / CK;
+  int ks = 1;
+  double best = 1e300;
+  for (int c = 1; c <= WQ_GEMM_MAX_SPLIT; c *= 2) {
+    if (c > 1 && kc / c < WQ_GEMM_MIN_STAGES) break;
+    const int slots = cluster_slots<BITS>(dev, c, smem);
+    if (slots <= 0) break;
+    const double waves = double((tiles + slots - 1) / slots);
+    const double t = waves * (double(kc) / c + kWaveStages + kSplitStages * (c - 1));
+    if (t < best - 1e-9) {
+      best = t;
+      ks = c;
+    }
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(unsigned((N + BN - 1) / BN), unsigned((M + BM - 1) / BM), unsigned(ks));
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = unsigned(ks);
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BITS>, tx, tc, scales, zeros, M, N, K, g,
+                            FastDiv(uint32_t(g / 32)), y);
 }
 
 }  // namespace

@@ -31,6 +31,41 @@ struct FastDiv {
   }
 };
 
+// ---- unpacking a 32-code unit with one AND per code ---------------------
+// A code q at bit p of a 32-bit word, with every other bit cleared, is the
+// subnormal float q * 2^(p-149) (no exponent bits, no implicit one).  Codes
+// above bit 23 - b are first brought down by one shift shared by the word
+// (a funnel shift for the 3-bit codes that straddle two words).
+// Position p (after its shift) of code i of a unit, and whether it needs the
+// shifted view.  Host-and-device so the lane's x scale can use it at run time.
+template <int BITS>
+__host__ __device__ constexpr int code_p(int i) {
+  const int P = (BITS * i) % 32;
+  if (P + BITS <= 23) return P;
+  return P - (BITS == 2 ? 10 : BITS == 8 ? 16 : 12);
+}
+template <int BITS>
+__host__ __device__ constexpr bool code_shifted(int i) {
+  return (BITS * i) % 32 + BITS > 23;
+}
+
+template <int BITS, int I>
+__device__ __forceinline__ float code_subnormal(const uint32_t (&w)[BITS]) {
+  constexpr int a = (BITS * I) / 32;
+  constexpr int p = code_p<BITS>(I);
+  constexpr uint32_t mask = ((1u << BITS) - 1u) << p;
+  uint32_t v;
+  if constexpr (!code_shifted<BITS>(I)) {
+    v = w[a];
+  } else if constexpr (BITS == 3) {
+    v = (a < 2) ? __funnelshift_r(w[a], w[a + 1 < 3 ? a + 1 : 2], 12) : (w[a] >> 12);
+  } else {
+    v = w[a] >> (BITS == 2 ? 10 : BITS == 8 ? 16 : 12);
+  }
+  return __uint_as_float(v & mask);
+}
+
+
 // ---- launchers (arguments already validated by the C ABI layer) ----------
 cudaError_t launch_quantize(const __half* W, int64_t N, int64_t K, int bits, int64_t g,
                             uint32_t* codes, __half* scales, __half* zeros, cudaStream_t st);

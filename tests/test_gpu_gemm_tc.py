@@ -29,7 +29,9 @@ def _run(Wh, x, bits, group):
 @pytest.mark.parametrize("bits", BITS)
 @pytest.mark.parametrize("M,N,K,group", [
     (17, 256, 128, 128), (64, 300, 384, 32), (256, 256, 256, 0), (257, 200, 640, 128),
-    (520, 513, 384, 64)])
+    (520, 513, 384, 64),
+    # few output tiles and a long K: split-K over a cluster of CTAs
+    (300, 520, 4096, 128), (40, 256, 2048, 0)])
 def test_tc_small(bits, M, N, K, group):
     Wh = wq_inputs.weight_f16(8, bits, N, K)
     x = wq_inputs.activations_bf16(8, M, M, K)
