@@ -10,10 +10,13 @@ import torch
 import oracle
 import wq_inputs
 
-# Per-element bound on |y_gpu - y_exact|: relative to sum_k |x w'|, plus an
-# absolute floor (the accuracy contract of wq_gemm).
+# Per-element bound on |y_gpu - y_exact| (the accuracy contract of wq_gemm):
+# the arithmetic before the output rounding may err by REL_TOL * sum_k |x w'|
+# plus an absolute floor, and y itself is bf16, whose round-to-nearest adds up
+# to 2^-8 |y| even when every earlier step is exact.
 REL_TOL = 2e-3
 ABS_TOL = 1e-3
+OUT_ROUND = 2.0 ** -8
 
 
 def wq():
@@ -40,7 +43,7 @@ def oracle_quantize(Wh: np.ndarray, bits: int, group: int):
 
 def assert_y_close(y_gpu: np.ndarray, y_ref: np.ndarray, bound: np.ndarray, what: str = ""):
     err = np.abs(y_gpu.astype(np.float64) - y_ref)
-    lim = REL_TOL * bound + ABS_TOL
+    lim = REL_TOL * bound + OUT_ROUND * np.abs(y_ref) + ABS_TOL
     bad = err > lim
     if bad.any():
         i = np.argwhere(bad)[0]
