@@ -114,7 +114,8 @@ wq_status wq_quantize_rtn(const void* W_f16, int64_t N, int64_t K, int bits, int
  * batch rows at a time.  Accuracy: every product is exact or rounded once
  * (w' to bf16 on the tensor-core path with grouped grids), sums are fp32, and
  * y carries one bf16 rounding (up to 2^-8 |y|); on realistic inputs each y
- * element lies within 2e-3 * sum_k |x w'| + 1e-3 of the exact value, which is
+ * element lies within 2e-3 * sum_k |x w'| + 2^-8 |y| + 1e-3 of the exact
+ * value (arithmetic error, the output rounding, an absolute floor), which is
  * the acceptance bound the tests use.  |x| must stay below 2^63.
  */
 wq_status wq_gemm(const void* x_bf16, int64_t M, int64_t N, int64_t K, const uint32_t* codes,

@@ -572,9 +572,9 @@ cudaError_t launch_bits(const __nv_bfloat16* x, int64_t M, int64_t N, int64_t K,
                         int64_t g, __nv_bfloat16* y, cudaStream_t st) {
   alignas(64) CUtensorMap tx, tc;
   if (!make_tensor_map_2d(&tx, TmaType::kBF16, x, uint64_t(K), uint64_t(M), uint64_t(K) * 2, BK, BM,
-                          true) ||
+                          128) ||
       !make_tensor_map_2d(&tc, TmaType::kU32, codes, uint64_t(K * BITS / 32), uint64_t(N),
-                          uint64_t(K * BITS / 8), CK * BITS / 32, BN, false))
+                          uint64_t(K * BITS / 8), CK * BITS / 32, BN, 0))
     return cudaErrorInvalidValue;
   constexpr uint32_t smem = TcCfg<BITS>::kSmem;
   static bool attr_set[64] = {};

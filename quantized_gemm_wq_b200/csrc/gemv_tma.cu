@@ -416,7 +416,7 @@ cudaError_t launch_bits(const __nv_bfloat16* x, int64_t N, int64_t K, const uint
   using Cfg = M1Cfg<BITS>;
   alignas(64) CUtensorMap tm;
   if (!make_tensor_map_2d(&tm, TmaType::kU32, codes, uint64_t(K * BITS / 32), uint64_t(N),
-                          uint64_t(K * BITS / 8), 32, 32, true))
+                          uint64_t(K * BITS / 8), 32, 32, 128))
     return cudaErrorInvalidValue;
   static bool attr_set[64] = {};
   int dev = 0;

@@ -27,18 +27,26 @@ EncodeTiledFn encode_fn() {
 }  // namespace
 
 bool make_tensor_map_2d(void* map, TmaType type, const void* base, uint64_t inner, uint64_t outer,
-                        uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, bool swizzle128) {
+                        uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, int swizzle_bytes) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   const cuuint64_t dims[2] = {inner, outer};
   const cuuint64_t strides[1] = {row_bytes};
   const cuuint32_t box[2] = {box_inner, box_outer};
   const cuuint32_t es[2] = {1, 1};
+  CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_NONE;
+  switch (swizzle_bytes) {
+    case 0: break;
+    case 32: swz = CU_TENSOR_MAP_SWIZZLE_32B; break;
+    case 64: swz = CU_TENSOR_MAP_SWIZZLE_64B; break;
+    case 128: swz = CU_TENSOR_MAP_SWIZZLE_128B; break;
+    default: return false;
+  }
   CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_UINT32;
   if (type == TmaType::kBF16) dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   return enc(static_cast<CUtensorMap*>(map), dt, 2, const_cast<void*>(base), dims, strides, box, es,
              CU_TENSOR_MAP_INTERLEAVE_NONE,
-             swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+             swz,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 

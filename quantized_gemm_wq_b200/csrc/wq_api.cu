@@ -112,23 +112,29 @@ wq_status wq_gemm(const void* x_bf16, int64_t M, int64_t N, int64_t K, const uin
   if (M > wq::kGemvMaxM && wq::gemm_tc_supported(K, bits)) {
     e = wq::launch_gemm_tc(x, M, N, K, codes, s, z, bits, g, y, strm);
   } else {
-    // Small batches, and K that the tensor-core path cannot stage with TMA
-    // (K not a multiple of 128): the GEMV, 16 batch rows per launch.
+    // Small batches, and K that the tensor-core GEMM cannot stage with TMA
+    // (K not a multiple of 128): 16 batch rows per launch.  One row runs the
+    // CUDA-core GEMV (its short pipeline wins at one row); 2..16 rows the
+    // tensor-core GEMV where its shape rules allow, else the CUDA-core GEMV.
     e = cudaSuccess;
     for (int64_t m0 = 0; m0 < M && e == cudaSuccess; m0 += wq::kGemvMaxM) {
       const int mc = int(M - m0 < wq::kGemvMaxM ? M - m0 : wq::kGemvMaxM);
-      e = wq::launch_gemv(x + m0 * K, mc, N, K, codes, s, z, bits, g, y + m0 * N, strm);
+      if (wq::gemv_tc_supported(mc, K, bits, g))
+        e = wq::launch_gemv_tc(x + m0 * K, mc, N, K, codes, s, z, bits, g, y + m0 * N, strm);
+      else
+        e = wq::launch_gemv(x + m0 * K, mc, N, K, codes, s, z, bits, g, y + m0 * N, strm);
     }
   }
   return e == cudaSuccess ? WQ_OK : WQ_ERR_CUDA;
 }
 
 wq_status wq_last_device_error(void) {
-  cudaError_t e1 = cudaSuccess, e2 = cudaSuccess;
+  cudaError_t e1 = cudaSuccess, e2 = cudaSuccess, e3 = cudaSuccess;
   const bool hit1 = wq::gemm_tc_read_and_clear_timeout(&e1);
   const bool hit2 = wq::gemv_m1_tma_read_and_clear_timeout(&e2);
-  if (e1 != cudaSuccess || e2 != cudaSuccess) return WQ_ERR_CUDA;
-  return (hit1 || hit2) ? WQ_ERR_DEVICE_TIMEOUT : WQ_OK;
+  const bool hit3 = wq::gemv_tc_read_and_clear_timeout(&e3);
+  if (e1 != cudaSuccess || e2 != cudaSuccess || e3 != cudaSuccess) return WQ_ERR_CUDA;
+  return (hit1 || hit2 || hit3) ? WQ_ERR_DEVICE_TIMEOUT : WQ_OK;
 }
 
 }  // extern "C"

@@ -88,6 +88,14 @@ cudaError_t launch_gemm_tc(const __nv_bfloat16* x, int64_t M, int64_t N, int64_t
                            const uint32_t* codes, const __half* scales, const __half* zeros,
                            int bits, int64_t g, __nv_bfloat16* y, cudaStream_t st);
 
+// Tensor-core decode GEMV (gemv_tc.cu): 2 <= M <= 16, K % 128 == 0, and for
+// 3-bit codes groups that are whole multiples of 128.
+bool gemv_tc_supported(int M, int64_t K, int bits, int64_t g);
+cudaError_t launch_gemv_tc(const __nv_bfloat16* x, int M, int64_t N, int64_t K,
+                           const uint32_t* codes, const __half* scales, const __half* zeros,
+                           int bits, int64_t g, __nv_bfloat16* y, cudaStream_t st);
+bool gemv_tc_read_and_clear_timeout(cudaError_t* err);
+
 // Reads and clears the device-side "bounded wait expired" flags of the current
 // device (synchronises the device).  Returns true if one was set.
 bool gemm_tc_read_and_clear_timeout(cudaError_t* err);
@@ -95,6 +103,6 @@ bool gemm_tc_read_and_clear_timeout(cudaError_t* err);
 // TMA tensor maps (a CUtensorMap is 128 bytes, 64-byte aligned).
 enum class TmaType { kU32, kBF16 };
 bool make_tensor_map_2d(void* map, TmaType type, const void* base, uint64_t inner, uint64_t outer,
-                        uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, bool swizzle128);
+                        uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, int swizzle_bytes);
 
 }  // namespace wq

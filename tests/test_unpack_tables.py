@@ -1,0 +1,71 @@
+"""The tensor-core GEMV's unpack tables (host data of the CUDA path, checked on
+the CPU): every AND of a table must pull exactly the codes it names out of a
+segment packed by the oracle's packer, each code once, in the low byte of its
+16-bit half (where bf16 bit patterns are linear in value)."""
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "quantized_gemm_wq_b200", "csrc", "unpack_tables.h")
+
+
+def parse_tables():
+    text = open(HEADER).read()
+    out = {}
+    for bits, body in re.findall(r"kUnpack(\d)\[64\] = \{(.*?)\};", text, re.S):
+        ops = re.findall(r"\{(\d+), 0x([0-9A-F]+)u, (\d+), (\d+), (\d+), (\d+)\}", body)
+        out[int(bits)] = [(int(s), int(m, 16), int(a), int(b), int(c), int(d)) for s, m, a, b, c, d in ops]
+    return out
+
+
+def test_header_is_generated():
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "gen_unpack_tables", os.path.join(ROOT, "quantized_gemm_wq_b200", "gen_unpack_tables.py"))
+    gen = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(gen)
+    assert open(HEADER).read() == gen.render()
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+def test_ops_extract_each_code_once(bits):
+    ops = parse_tables()[bits]
+    assert len(ops) == 64
+    seen = sorted([o[2] for o in ops] + [o[4] for o in ops])
+    assert seen == list(range(128))
+    rng = np.random.default_rng(bits)
+    for trial in range(20):
+        q = rng.integers(0, 1 << bits, size=(1, 128), dtype=np.uint8)
+        if trial == 0:
+            q[:] = (1 << bits) - 1                      # all bits set: masks must not leak
+        words = oracle.pack(q, bits)[0]
+        stream = 0
+        for i, w in enumerate(words):
+            stream |= int(w) << (32 * i)
+        for s, m, lo, blo, hi, bhi in ops:
+            assert blo + bits <= 8 and bhi + bits <= 8
+            assert m == ((((1 << bits) - 1) << blo) | ((((1 << bits) - 1) << bhi) << 16))
+            v = ((stream >> s) & 0xFFFFFFFF) & m
+            assert v & 0xFFFF == int(q[0, lo]) << blo
+            assert v >> 16 == int(q[0, hi]) << bhi
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+def test_bf16_patterns_are_linear(bits):
+    """Pattern p < 0x100 in a bf16 is p 2^-133, so code << b reads as q 2^(b-133)."""
+    for p in range(256):
+        f = np.array([p << 16], dtype=np.uint32).view(np.float32)[0]
+        assert float(f) == p * 2.0 ** -133
+
+
+def test_shift_counts():
+    t = parse_tables()
+    # windows needing a shift (start not on a word boundary)
+    shifts = {b: len({o[0] for o in ops if o[0] % 32}) for b, ops in t.items()}
+    assert shifts[2] == 8 and shifts[4] == 16 and shifts[8] == 32
+    assert shifts[3] <= 28
