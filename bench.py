@@ -464,17 +464,19 @@ def main(argv=None):
 def run_case(case: str) -> None:
     """One small profiling case (for ncu): ``decode`` runs one decode step of
     the headline layer (the four M = 1 GEMV launches, after 3 warm-up steps);
-    ``gemv:<linear index>`` one M = 1 GEMV of that projection; ``prefill:<linear
-    index>`` one prefill GEMM (M = 2048) of the Llama-13B-shaped workload."""
+    ``gemv:<linear index>`` one M = 1 GEMV of that projection; ``gemv16:<linear
+    index>`` the same with a batch of 16 rows (the tensor-core GEMV);
+    ``prefill:<linear index>`` one prefill GEMM (M = 2048) of the
+    Llama-13B-shaped workload."""
     import torch
     import quantized_gemm_wq_b200 as wq
     kind, _, arg = case.partition(":")
     wl = PREFILL if kind == "prefill" else HEADLINE
     w = wq_inputs.WORKLOADS[wl]
     lins = list(enumerate(w["linears"]))
-    if kind in ("gemv", "prefill"):
+    if kind in ("gemv", "gemv16", "prefill"):
         lins = [lins[int(arg or 0)]]
-    M = w["Ms"][0] if kind == "prefill" else 1
+    M = w["Ms"][0] if kind == "prefill" else (16 if kind == "gemv16" else 1)
     ops = []
     for li, (name, N, K) in lins:
         W = torch.from_numpy(wq_inputs.weight_f16(0, li, N, K, dist=w["dist"])).cuda()

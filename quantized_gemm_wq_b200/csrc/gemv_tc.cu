@@ -81,7 +81,7 @@ struct TcvM {
   static constexpr uint32_t kSegB = 16 * kChunk;            // B bytes per segment
   // Segments a CTA may own (its B operand stays resident); 8-bit code boxes
   // are twice as large, so they leave less room.
-  static constexpr int kMaxJ = MP == 4 ? (BITS == 8 ? 16 : 32) : (BITS == 8 ? 4 : 8);
+  static constexpr int kMaxJ = MP == 4 ? (BITS == 8 ? 16 : 32) : (BITS == 8 ? 4 : 11);
   static constexpr uint32_t kBBytes = kMaxJ * kSegB + 256;  // + what rows past MP may read
   static constexpr uint32_t kXsBytes = kMaxJ * 4 * MP * 4;  // 2^-69 sum(x) per segment, AU, row
 };
