@@ -58,10 +58,14 @@ constexpr uint64_t kDrainNs = 200000000ull;      // 0.2 s for the exit path
 
 template <int BITS>
 struct TcCfg {
-  static constexpr int kStages = BITS == 8 ? 2 : 3;        // x / W' ring
+  // The x ring is the deep one (its TMA loads must cover the L2/HBM latency);
+  // W' is written by the dequantising warps just ahead of the MMAs.
+  static constexpr int kXStages = BITS == 8 ? 3 : 4;       // x ring (64 K each)
+  static constexpr int kWStages = 2;                       // W' ring (64 K each)
   static constexpr int kCStages = 2;                       // codes ring (128 K each)
   static constexpr uint32_t kCBytes = uint32_t(BN) * CK * BITS / 8;
-  static constexpr uint32_t kRingBytes = kStages * (kABytes + kBBytes) + kCStages * kCBytes;
+  static constexpr uint32_t kRingBytes =
+      kXStages * kABytes + kWStages * kBBytes + kCStages * kCBytes;
   static constexpr uint32_t kSmem = kRingBytes + 1024 + 256 + 4 * BN;
 };
 static_assert(TcCfg<4>::kSmem <= 232448, "shared memory");
@@ -257,17 +261,18 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                int64_t N, int64_t K, int64_t g, FastDiv units_per_group,
                __nv_bfloat16* __restrict__ y) {
   using Cfg = TcCfg<BITS>;
-  constexpr int S = Cfg::kStages, SC = Cfg::kCStages;
+  constexpr int SX = Cfg::kXStages, SW = Cfg::kWStages, SC = Cfg::kCStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sA = base;                                   // [S][256 x 64 bf16], swizzled
-  uint8_t* sB = sA + S * kABytes;                       // [S][256 x 64 bf16], swizzled
-  uint8_t* sC = sB + S * kBBytes;                       // [SC][256 x 128 codes]
+  uint8_t* sA = base;                                   // [SX][256 x 64 bf16], swizzled
+  uint8_t* sB = sA + SX * kABytes;                      // [SW][256 x 64 bf16], swizzled
+  uint8_t* sC = sB + SW * kBBytes;                      // [SC][256 x 128 codes]
   uint64_t* bars = reinterpret_cast<uint64_t*>(sC + SC * Cfg::kCBytes);
   uint64_t* full_a = bars;             // TMA x landed            (1 arrival + bytes)
-  uint64_t* full_b = full_a + S;       // W' written             (kDqWarps arrivals)
-  uint64_t* empty_ab = full_b + S;     // MMAs done with stage   (commit)
-  uint64_t* full_c = empty_ab + S;     // TMA codes landed       (1 arrival + bytes)
+  uint64_t* empty_a = full_a + SX;     // MMAs done with x slot   (commit)
+  uint64_t* full_b = empty_a + SX;     // W' written             (kDqWarps arrivals)
+  uint64_t* empty_b = full_b + SW;     // MMAs done with W' slot (commit)
+  uint64_t* full_c = empty_b + SW;     // TMA codes landed       (1 arrival + bytes)
   uint64_t* empty_c = full_c + SC;     // codes consumed         (kDqWarps arrivals)
   uint64_t* tmem_full = empty_c + SC;  // accumulators final     (commit)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tmem_full + 1);
@@ -288,10 +293,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
   const bool rowwise = (g == K);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < S; ++s) {
+    for (int s = 0; s < SX; ++s) {
       mbar_init(&full_a[s], 1);
+      mbar_init(&empty_a[s], 1);
+    }
+    for (int s = 0; s < SW; ++s) {
       mbar_init(&full_b[s], kDqWarps);
-      mbar_init(&empty_ab[s], 1);
+      mbar_init(&empty_b[s], 1);
     }
     for (int s = 0; s < SC; ++s) {
       mbar_init(&full_c[s], 1);
@@ -328,16 +336,16 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
           tma_load_2d(sC + cs * Cfg::kCBytes, &tm_c, &full_c[cs], (kt >> 1) * (CK * BITS / 32), int(n0));
           ++issued_c;
         }
-        const int s = j % S;
-        if (j >= S) ok = mbar_wait(&empty_ab[s], ((j / S) - 1) & 1, abort);
+        const int s = j % SX;
+        if (j >= SX) ok = mbar_wait(&empty_a[s], ((j / SX) - 1) & 1, abort);
         if (!ok) break;
         mbar_expect_tx(&full_a[s], kABytes);
         tma_load_2d(sA + s * kABytes, &tm_x, &full_a[s], kt * BK, int(m0));
         ++issued_a;
       }
       if (!ok) {   // let the copies still in flight land before shared memory goes away
-        for (int kt = (issued_a > S ? issued_a - S : 0); kt < issued_a; ++kt)
-          mbar_drain(&full_a[kt % S], (kt / S) & 1);
+        for (int kt = (issued_a > SX ? issued_a - SX : 0); kt < issued_a; ++kt)
+          mbar_drain(&full_a[kt % SX], (kt / SX) & 1);
         for (int c = (issued_c > SC ? issued_c - SC : 0); c < issued_c; ++c)
           mbar_drain(&full_c[c % SC], (c / SC) & 1);
       }
@@ -347,13 +355,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
     if (lane == 0) {
       bool ok = true;
       for (int kt = kt0; kt < kt1 && ok; ++kt) {
-        const int s = (kt - kt0) % S;
-        const uint32_t par = ((kt - kt0) / S) & 1;
-        ok = mbar_wait(&full_a[s], par, abort) && mbar_wait(&full_b[s], par, abort);
+        const int j = kt - kt0;
+        const int sx = j % SX, sw = j % SW;
+        ok = mbar_wait(&full_a[sx], (j / SX) & 1, abort) && mbar_wait(&full_b[sw], (j / SW) & 1, abort);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t a0 = smem_u32(sA + s * kABytes);
-        const uint32_t b0 = smem_u32(sB + s * kBBytes);
+        const uint32_t a0 = smem_u32(sA + sx * kABytes);
+        const uint32_t b0 = smem_u32(sB + sw * kBBytes);
 #pragma unroll
         for (int kk = 0; kk < BK / kMmaK; ++kk) {
           const uint64_t bd = sw128_desc(b0 + kk * kMmaK * 2);
@@ -363,7 +371,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
             umma(tmem + uint32_t(mt * kMmaN), ad, bd, (kt > kt0 || kk > 0) ? 1u : 0u);
           }
         }
-        umma_commit(&empty_ab[s]);
+        umma_commit(&empty_a[sx]);
+        umma_commit(&empty_b[sw]);
       }
       umma_commit(tmem_full);      // always: the teardown waits on it before freeing TMEM
     }
@@ -382,35 +391,46 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
     // code comes out of one AND as the subnormal float q 2^(p-149), one FMUL by
     // 2^(119-p) (exact) gives q 2^-30, and the FMA is exact (s q and s z have at
     // most 20 significant bits); the bf16 conversion is the only rounding.
-    // Scale and zero of the next step are loaded one step ahead.
+    // Scale and zero of the next step are loaded one step ahead as raw fp16
+    // bits; nothing reads those registers until that step (a use right after
+    // the load would stall the warp for the whole load latency), so the loop
+    // runs two steps per iteration with two register sets.
     const int r0 = 32 * dw + (lane >> 1);
-    auto load_ab = [&](int kt, float (&A)[2], float (&B)[2]) {
+    const unsigned short* sh = reinterpret_cast<const unsigned short*>(scales);
+    const unsigned short* zh = reinterpret_cast<const unsigned short*>(zeros);
+    auto load_raw = [&](int kt, uint16_t (&s2)[2], uint16_t (&z2)[2]) {
       const int64_t k = int64_t(kt) * BK + 32 * cu;
-      const uint32_t grp = units_per_group.div(uint32_t(k >> 5));
+      const uint32_t grp = units_per_group.div(uint32_t(k < K ? k >> 5 : 0));
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
         const int64_t n = n0 + r0 + 16 * i;
-        A[i] = 0.0f;
-        B[i] = 0.0f;
+        s2[i] = 0;
+        z2[i] = 0;
         if (kt < kt1 && n < N && k < K) {
-          const float sc = rowwise ? 1.0f : __half2float(scales[n * G + grp]);
-          A[i] = sc * 0x1p30f;
-          B[i] = -sc * __half2float(zeros[n * G + grp]);
+          s2[i] = rowwise ? uint16_t(0x3C00) : __ldg(sh + n * G + grp);   // 0x3C00: fp16 1.0
+          z2[i] = __ldg(zh + n * G + grp);
         }
       }
     };
-    float A[2], B[2];
-    load_ab(kt0, A, B);
     bool ok = true;
-    for (int kt = kt0; kt < kt1 && ok; ++kt) {
+    // One K step with the step's raw scale/zero (cs, cz); the next step's are
+    // requested into (ns, nz).
+    auto step = [&](int kt, const uint16_t (&cs2)[2], const uint16_t (&cz2)[2], uint16_t (&ns2)[2],
+                    uint16_t (&nz2)[2]) {
+      load_raw(kt + 1, ns2, nz2);
+      float A[2], B[2];
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const float sc = __half2float(__ushort_as_half(cs2[i]));
+        A[i] = sc * 0x1p30f;
+        B[i] = -sc * __half2float(__ushort_as_half(cz2[i]));
+      }
       const int j = kt - kt0;
-      const int c = j >> 1, cs = c % SC, s = j % S;
-      float An[2], Bn[2];
-      load_ab(kt + 1, An, Bn);
+      const int c = j >> 1, cs = c % SC, s = j % SW;
       ok = mbar_wait(&full_c[cs], (c / SC) & 1, abort);
-      if (ok && j >= S) ok = mbar_wait(&empty_ab[s], ((j / S) - 1) & 1, abort);
+      if (ok && j >= SW) ok = mbar_wait(&empty_b[s], ((j / SW) - 1) & 1, abort);
       ok = __all_sync(0xffffffffu, ok);      // the warp leaves the loop together
-      if (!ok) break;
+      if (!ok) return;
       const uint8_t* ctile = sC + cs * Cfg::kCBytes;
       uint8_t* btile = sB + s * kBBytes;
       const int ucode = (kt & 1) * 2 + cu;   // unit index within the 128-code stage
@@ -423,9 +443,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         DqPairs<BITS, 0>::run(w, A[i], B[i], p);
         uint8_t* brow = btile + r * 128;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int chunk = (cu * 4 + j) ^ (r & 7);
-          *reinterpret_cast<uint4*>(brow + chunk * 16) = make_uint4(p[4 * j], p[4 * j + 1], p[4 * j + 2], p[4 * j + 3]);
+        for (int jj = 0; jj < 4; ++jj) {
+          const int chunk = (cu * 4 + jj) ^ (r & 7);
+          *reinterpret_cast<uint4*>(brow + chunk * 16) = make_uint4(p[4 * jj], p[4 * jj + 1], p[4 * jj + 2], p[4 * jj + 3]);
         }
       }
       fence_async_smem();
@@ -434,11 +454,12 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         mbar_arrive(&full_b[s]);
         if ((j & 1) || kt == kt1 - 1) mbar_arrive(&empty_c[cs]);
       }
-#pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        A[i] = An[i];
-        B[i] = Bn[i];
-      }
+    };
+    uint16_t s0r[2], z0r[2], s1r[2], z1r[2];
+    load_raw(kt0, s0r, z0r);
+    for (int kt = kt0; kt < kt1 && ok; kt += 2) {
+      step(kt, s0r, z0r, s1r, z1r);
+      if (ok && kt + 1 < kt1) step(kt + 1, s1r, z1r, s0r, z0r);
     }
     if (ok) ok = mbar_wait(tmem_full, 0, abort);
     ep_ok = __all_sync(0xffffffffu, ok);     // tcgen05.ld needs the whole warp
