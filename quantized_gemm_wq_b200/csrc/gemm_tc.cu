@@ -396,28 +396,38 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
     // the load would stall the warp for the whole load latency), so the loop
     // runs two steps per iteration with two register sets.
     const int r0 = 32 * dw + (lane >> 1);
-    const unsigned short* sh = reinterpret_cast<const unsigned short*>(scales);
-    const unsigned short* zh = reinterpret_cast<const unsigned short*>(zeros);
+    // This thread's two rows of the scale and zero arrays (row n >= N: none).
+    const unsigned short* srow[2];
+    const unsigned short* zrow[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int64_t n = n0 + r0 + 16 * i;
+      srow[i] = n < N ? reinterpret_cast<const unsigned short*>(scales) + n * G : nullptr;
+      zrow[i] = n < N ? reinterpret_cast<const unsigned short*>(zeros) + n * G : nullptr;
+    }
     auto load_raw = [&](int kt, uint16_t (&s2)[2], uint16_t (&z2)[2]) {
-      const int64_t k = int64_t(kt) * BK + 32 * cu;
+      const int k = kt * BK + 32 * cu;
       const uint32_t grp = units_per_group.div(uint32_t(k < K ? k >> 5 : 0));
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
-        const int64_t n = n0 + r0 + 16 * i;
         s2[i] = 0;
         z2[i] = 0;
-        if (kt < kt1 && n < N && k < K) {
-          s2[i] = rowwise ? uint16_t(0x3C00) : __ldg(sh + n * G + grp);   // 0x3C00: fp16 1.0
-          z2[i] = __ldg(zh + n * G + grp);
+        if (kt < kt1 && srow[i] != nullptr && k < K) {
+          s2[i] = rowwise ? uint16_t(0x3C00) : __ldg(srow[i] + grp);   // 0x3C00: fp16 1.0
+          z2[i] = __ldg(zrow[i] + grp);
         }
       }
     };
+    // With groups that are whole multiples of 128 the two K steps of a pair
+    // (kt - kt0 even, and kt + 1) use one group, so a pair loads its scale and
+    // zero once, during its second step, for the next pair.
+    const bool pair_group = (g % (2 * BK)) == 0;
     bool ok = true;
     // One K step with the step's raw scale/zero (cs, cz); the next step's are
     // requested into (ns, nz).
     auto step = [&](int kt, const uint16_t (&cs2)[2], const uint16_t (&cz2)[2], uint16_t (&ns2)[2],
-                    uint16_t (&nz2)[2]) {
-      load_raw(kt + 1, ns2, nz2);
+                    uint16_t (&nz2)[2], bool load_next) {
+      if (load_next) load_raw(kt + 1, ns2, nz2);
       float A[2], B[2];
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
@@ -457,9 +467,18 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
     };
     uint16_t s0r[2], z0r[2], s1r[2], z1r[2];
     load_raw(kt0, s0r, z0r);
-    for (int kt = kt0; kt < kt1 && ok; kt += 2) {
-      step(kt, s0r, z0r, s1r, z1r);
-      if (ok && kt + 1 < kt1) step(kt + 1, s1r, z1r, s0r, z0r);
+    if (pair_group) {
+      for (int kt = kt0; kt < kt1 && ok; kt += 4) {   // two pairs: register sets 0 then 1
+        step(kt, s0r, z0r, s1r, z1r, false);
+        if (ok && kt + 1 < kt1) step(kt + 1, s0r, z0r, s1r, z1r, true);
+        if (ok && kt + 2 < kt1) step(kt + 2, s1r, z1r, s0r, z0r, false);
+        if (ok && kt + 3 < kt1) step(kt + 3, s1r, z1r, s0r, z0r, true);
+      }
+    } else {
+      for (int kt = kt0; kt < kt1 && ok; kt += 2) {
+        step(kt, s0r, z0r, s1r, z1r, true);
+        if (ok && kt + 1 < kt1) step(kt + 1, s1r, z1r, s0r, z0r, true);
+      }
     }
     if (ok) ok = mbar_wait(tmem_full, 0, abort);
     ep_ok = __all_sync(0xffffffffu, ok);     // tcgen05.ld needs the whole warp
