@@ -37,10 +37,9 @@ namespace {
 
 constexpr int kScaleS = 64;
 
-// Resident CTAs per SM the register budget is sized for.
-#ifndef WQ_GEMV_M1_MIN_CTAS
-#define WQ_GEMV_M1_MIN_CTAS 2
-#endif
+// Resident CTAs per SM the register budget is sized for: 2, or 3 for grids
+// that would otherwise need a second wave of 2 per SM (2..4 bits; 8-bit
+// stages are too large for a third CTA).
 // Split-K heuristic: CTAs wanted in total, and K stages kept per CTA.
 #ifndef WQ_GEMV_M1_TARGET_CTAS
 #define WQ_GEMV_M1_TARGET_CTAS 444
@@ -206,8 +205,8 @@ __device__ __forceinline__ void load_unit_at(uint32_t stage, const uint32_t (&o)
 // warps 0..NW-1 consume: warp w takes units 4w..4w+3 of every box, lane l
 // rows lr, lr+8, lr+16, lr+24 (lr = l % 8) of unit 4w + l / 8.  A stage is
 // released when every consumer warp has arrived on its "empty" barrier.
-template <int BITS>
-__global__ void __launch_bounds__(32 * (M1Cfg<BITS>::NW + 1), WQ_GEMV_M1_MIN_CTAS)
+template <int BITS, int MINB>
+__global__ void __launch_bounds__(32 * (M1Cfg<BITS>::NW + 1), MINB)
 gemv_m1_tma_kernel(const __grid_constant__ CUtensorMap tm_codes, const __nv_bfloat16* __restrict__ x,
                    int64_t N, int64_t K, const __half* __restrict__ scales,
                    const __half* __restrict__ zeros, FastDiv units_per_group,
@@ -419,11 +418,16 @@ cudaError_t launch_bits(const __nv_bfloat16* x, int64_t N, int64_t K, const uint
                           uint64_t(K * BITS / 8), 32, 32, 128))
     return cudaErrorInvalidValue;
   static bool attr_set[64] = {};
+  static int sms[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    const cudaError_t e = cudaFuncSetAttribute(gemv_m1_tma_kernel<BITS>,
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
+    cudaError_t e = cudaFuncSetAttribute(gemv_m1_tma_kernel<BITS, 2>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
+    if (e == cudaSuccess && BITS != 8)
+      e = cudaFuncSetAttribute(gemv_m1_tma_kernel<BITS, BITS == 8 ? 2 : 3>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
@@ -448,7 +452,13 @@ cudaError_t launch_bits(const __nv_bfloat16* x, int64_t N, int64_t K, const uint
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, gemv_m1_tma_kernel<BITS>, tm, x, N, K, scales, zeros, upg, y);
+  // A grid between two and three CTAs per SM runs in one wave with the
+  // variant sized for three.
+  const int64_t ctas = tiles * ks, nsm = (dev >= 0 && dev < 64) ? sms[dev] : 0;
+  if (BITS != 8 && ctas > 2 * nsm && ctas <= 3 * nsm)
+    return cudaLaunchKernelEx(&cfg, gemv_m1_tma_kernel<BITS, BITS == 8 ? 2 : 3>, tm, x, N, K, scales,
+                              zeros, upg, y);
+  return cudaLaunchKernelEx(&cfg, gemv_m1_tma_kernel<BITS, 2>, tm, x, N, K, scales, zeros, upg, y);
 }
 
 }  // namespace

@@ -30,6 +30,8 @@ def _run(Wh, x, bits, group):
 @pytest.mark.parametrize("M,N,K,group", [
     (17, 256, 128, 128), (64, 300, 384, 32), (256, 256, 256, 0), (257, 200, 640, 128),
     (520, 513, 384, 64),
+    # groups spanning several K-step pairs, and one that splits a pair
+    (96, 384, 1024, 256), (33, 130, 768, 384), (48, 200, 384, 96),
     # few output tiles and a long K: split-K over a cluster of CTAs
     (300, 520, 4096, 128), (40, 256, 2048, 0)])
 def test_tc_small(bits, M, N, K, group):
