@@ -368,7 +368,7 @@ cudaError_t launch_bits(const __nv_bfloat16* x, int M, int64_t N, int64_t K,
   const FastDiv upg(uint32_t(g / 32));
   auto grid_for = [&](int R) { return dim3(unsigned((N + int64_t(kWarps) * R - 1) / (int64_t(kWarps) * R))); };
   if (M <= 1) {
-    if (gemv_m1_tma_supported(K, BITS))   // rows start on 16 bytes: TMA-staged codes
+    if (gemv_m1_tma_supported(x, codes, K, BITS))   // TMA-staged codes and x
       return launch_gemv_m1_tma(x, N, K, codes, scales, zeros, BITS, g, y, st);
     constexpr int R = BITS == 8 ? 2 : 4;
     gemv1_kernel<BITS, R><<<grid_for(R), kThreads, 0, st>>>(x, N, K, codes, scales, zeros, upg, y);

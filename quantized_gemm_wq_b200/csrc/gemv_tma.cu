@@ -37,9 +37,8 @@ namespace {
 
 constexpr int kScaleS = 64;
 
-// Resident CTAs per SM the register budget is sized for: 2, or 3 for grids
-// that would otherwise need a second wave of 2 per SM (2..4 bits; 8-bit
-// stages are too large for a third CTA).
+// The kernel is compiled for 2 resident CTAs per SM, and for 3 for grids that
+// would otherwise need a second wave of 2 per SM.
 // Split-K heuristic: CTAs wanted in total, and K stages kept per CTA.
 #ifndef WQ_GEMV_M1_TARGET_CTAS
 #define WQ_GEMV_M1_TARGET_CTAS 444
@@ -51,26 +50,6 @@ constexpr uint64_t kWaitNs = 1000000000ull;
 
 __device__ unsigned int g_gemv_tma_timeout;
 
-#ifndef WQ_GEMV_PAIRS
-#define WQ_GEMV_PAIRS 0
-#endif
-
-__device__ __forceinline__ uint64_t pack_f2(float lo, float hi) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-  return r;
-}
-__device__ __forceinline__ uint64_t ffma_f2(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
-__device__ __forceinline__ float2 unpack_f2(uint64_t v) {
-  float lo, hi;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-  return make_float2(lo, hi);
-}
-
 // d[I % 4] += x'[I] * f_I for I = I0..31 (four independent chains).
 template <int BITS, int I>
 struct Dot {
@@ -80,17 +59,6 @@ struct Dot {
     if constexpr (I + 1 < 32) Dot<BITS, I + 1>::run(w, xp, d);
   }
 };
-// Same with packed f32x2 FMAs over code pairs (2 chains of pairs).
-template <int BITS, int J>
-struct Dot2 {
-  __device__ __forceinline__ static void run(const uint32_t (&w)[BITS], const uint64_t (&xp2)[16],
-                                             uint64_t (&d)[2]) {
-    d[J & 1] = ffma_f2(xp2[J], pack_f2(code_subnormal<BITS, 2 * J>(w), code_subnormal<BITS, 2 * J + 1>(w)),
-                       d[J & 1]);
-    if constexpr (J + 1 < 16) Dot2<BITS, J + 1>::run(w, xp2, d);
-  }
-};
-
 __device__ __forceinline__ uint32_t saddr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -148,8 +116,12 @@ struct M1Cfg {
   static constexpr int STAGE_WORDS = 32 * BITS;      // 32 units of one row
   static constexpr int BOX_BYTES = 32 * 128;         // one TMA box: 32 rows x 128 bytes, swizzled
   static constexpr int STAGE_BYTES = BITS * BOX_BYTES;
-  static constexpr int XS_BYTES = NW * 2 * 128 * 4;  // per warp: staged x', double-buffered
-  static constexpr int SMEM = D * STAGE_BYTES + XS_BYTES + 2 * D * 8 + 1024;
+  static constexpr int XRAW_BYTES = 1024 * 2;        // the stage's 1024 x values, bf16, as copied
+  static constexpr int XU = 36;                      // floats per staged unit of x' (32 + bank pad)
+  static constexpr int XS_BYTES = NW * 4 * XU * 4;   // per warp: x' of its 4 units
+  // ring, raw x slots, x' buffers and barriers; the scale table follows
+  static constexpr int FIXED = D * (STAGE_BYTES + XRAW_BYTES) + XS_BYTES + 2 * D * 8;
+  static int smem(int gcap) { return FIXED + 32 * gcap * 8 + 1024; }
 };
 
 // Shared-memory byte offset of word wi (0 .. 32*BITS-1) of row r in a stage:
@@ -200,27 +172,36 @@ __device__ __forceinline__ void load_unit_at(uint32_t stage, const uint32_t (&o)
   }
 }
 
-// One CTA: 32 output rows over the whole K.  Warp NW is the producer (one lane
-// issues the TMA copy of each 32-row x 32-unit box into a ring of D stages);
-// warps 0..NW-1 consume: warp w takes units 4w..4w+3 of every box, lane l
-// rows lr, lr+8, lr+16, lr+24 (lr = l % 8) of unit 4w + l / 8.  A stage is
-// released when every consumer warp has arrived on its "empty" barrier.
+// One CTA: 32 output rows over its share of K.  Warp NW is the producer: one
+// lane issues, per stage, the TMA copy of the 32-row x 32-unit box of codes and
+// a bulk copy of the stage's 1024 x values (bf16) into a ring of D stages,
+// both completing on the stage's "full" barrier.  Warps 0..NW-1 consume: warp
+// w takes units 4w..4w+3 of every box, lane l rows lr, lr+8, lr+16, lr+24
+// (lr = l % 8) of unit 4w + l / 8.  A stage is released when every consumer
+// warp has arrived on its "empty" barrier.  The scales and zeros of the CTA's
+// rows are read from global memory once, into a shared table of (s, z) pairs
+// covering up to gcap groups, while the first codes are in flight; a CTA whose
+// K range spans more groups reloads the table between stages.  The consumers
+// therefore wait on nothing but the ring.
 template <int BITS, int MINB>
 __global__ void __launch_bounds__(32 * (M1Cfg<BITS>::NW + 1), MINB)
 gemv_m1_tma_kernel(const __grid_constant__ CUtensorMap tm_codes, const __nv_bfloat16* __restrict__ x,
                    int64_t N, int64_t K, const __half* __restrict__ scales,
-                   const __half* __restrict__ zeros, FastDiv units_per_group,
+                   const __half* __restrict__ zeros, FastDiv units_per_group, int gcap,
                    __nv_bfloat16* __restrict__ y) {
   using Cfg = M1Cfg<BITS>;
-  constexpr int NW = Cfg::NW, D = Cfg::D;
+  constexpr int NW = Cfg::NW, D = Cfg::D, XU = Cfg::XU;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   __shared__ float red[NW][32];
   // the swizzle pattern repeats every 1024 bytes: align the ring to it
   uint8_t* smem = smem_raw + ((1024 - (saddr(smem_raw) & 1023)) & 1023);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t ring = saddr(smem);
-  const uint32_t full0 = saddr(smem + D * Cfg::STAGE_BYTES + Cfg::XS_BYTES);
+  const uint32_t xraw0 = ring + D * Cfg::STAGE_BYTES;
+  uint8_t* xs_base = smem + D * (Cfg::STAGE_BYTES + Cfg::XRAW_BYTES);
+  const uint32_t full0 = saddr(xs_base + Cfg::XS_BYTES);
   const uint32_t empty0 = full0 + 8 * D;
+  float2* tbl = reinterpret_cast<float2*>(xs_base + Cfg::XS_BYTES + 16 * D);
 
   const int64_t row0 = int64_t(blockIdx.x) * 32;
   const int64_t KU = K / 32;
@@ -241,16 +222,18 @@ gemv_m1_tma_kernel(const __grid_constant__ CUtensorMap tm_codes, const __nv_bflo
   }
   __syncthreads();
 
-  bool ok = true;
   if (warp == NW) {
     // ---------------------------------------------------------------- producer
     if (lane == 0) {
+      bool ok = true;
       for (int t = 0; t < T && ok; ++t) {
         const int s = t % D;
         if (t >= D) ok = mbar_wait_bounded(empty0 + 8 * s, uint32_t(((t / D) - 1) & 1));
         if (!ok) break;
+        const int64_t k0 = int64_t(tb + t) * 1024;
+        const uint32_t xbytes = uint32_t((K - k0 < 1024 ? K - k0 : 1024) * 2);
         asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(full0 + 8 * s),
-                     "r"(uint32_t(Cfg::STAGE_BYTES))
+                     "r"(uint32_t(Cfg::STAGE_BYTES) + xbytes)
                      : "memory");
 #pragma unroll
         for (int b = 0; b < BITS; ++b)
@@ -259,6 +242,11 @@ gemv_m1_tma_kernel(const __grid_constant__ CUtensorMap tm_codes, const __nv_bflo
               " [%0], [%1, {%3, %4}], [%2];" ::"r"(ring + s * Cfg::STAGE_BYTES + b * Cfg::BOX_BYTES),
               "l"(&tm_codes), "r"(full0 + 8 * s), "r"((tb + t) * Cfg::STAGE_WORDS + 32 * b), "r"(int(row0))
               : "memory");
+        asm volatile(
+            "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                xraw0 + s * Cfg::XRAW_BYTES),
+            "l"(x + k0), "r"(xbytes), "r"(full0 + 8 * s)
+            : "memory");
       }
       if (!ok) {   // copies issued but not consumed must land before the CTA exits
         for (int t = 0; t < T; ++t) {
@@ -271,84 +259,88 @@ gemv_m1_tma_kernel(const __grid_constant__ CUtensorMap tm_codes, const __nv_bflo
   } else {
     // ---------------------------------------------------------------- consumers
     const int lr = lane & 7, kq = lane >> 3;
-    float* xs = reinterpret_cast<float*>(smem + D * Cfg::STAGE_BYTES) + warp * 256;
+    float* xs = reinterpret_cast<float*>(xs_base) + warp * 4 * XU;
     const float xscale = __uint_as_float(uint32_t(127 + kScaleS - code_p<BITS>(lane)) << 23);
-    const bool rows_full = row0 + 32 <= N;
-    const __half* srow = scales + (row0 + lr) * G;
-    const __half* zrow = zeros + (row0 + lr) * G;
-    const int64_t G8 = 8 * G;
     const int ub = 4 * warp;                           // this warp's first unit in a box
 
-    // x of box t, position `lane` of this warp's 4 units.
-    auto load_x = [&](int t, float (&xv)[4]) {
-      const int64_t u0 = int64_t(tb + t) * 32 + ub;
-      const __nv_bfloat16* xc = x + u0 * 32 + lane;
-      if (t < T && u0 + 4 <= KU) {
+    // (s, z) of rows row0..row0+31, groups [wg0, wg0 + gcap): thread c of the
+    // 256 consumers reads groups c % 8, c % 8 + 8, ... of row c / 8.  Every
+    // consumer passes both barriers, also after a timed-out wait.
+    const int trow = threadIdx.x >> 3, tj = threadIdx.x & 7;
+    const bool trow_in = row0 + trow < N;
+    const __half* srow = scales + (trow_in ? row0 + trow : 0) * G;
+    const __half* zrow = zeros + (trow_in ? row0 + trow : 0) * G;
+    auto load_table = [&](int64_t wg0) {
+      float sv[16], zv[16];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) xv[u] = __bfloat162float(xc[32 * u]);
-      } else {
-#pragma unroll
-        for (int u = 0; u < 4; ++u) xv[u] = (t < T && u0 + u < KU) ? __bfloat162float(xc[32 * u]) : 0.0f;
+      for (int i = 0; i < 16; ++i) {
+        const int j = tj + 8 * i;
+        const bool in = trow_in && j < gcap && wg0 + j < G;
+        sv[i] = in ? __half2float(srow[wg0 + j]) : 0.0f;
+        zv[i] = in ? __half2float(zrow[wg0 + j]) : 0.0f;
       }
-    };
-    // stage x' of box t and return sum x of this lane's unit kq.
-    auto stage_x = [&](int t, const float (&xv)[4]) {
-      float* dst = xs + (t & 1) * 128;
+      asm volatile("bar.sync 1, %0;" ::"n"(32 * NW) : "memory");   // old table no longer read
 #pragma unroll
-      for (int u = 0; u < 4; ++u) dst[u * 32 + lane] = xv[u] * xscale;
-      const bool h16 = lane & 16, h8 = lane & 8;
-      float a = (h16 ? xv[2] : xv[0]) + __shfl_xor_sync(0xffffffffu, h16 ? xv[0] : xv[2], 16);
-      float b = (h16 ? xv[3] : xv[1]) + __shfl_xor_sync(0xffffffffu, h16 ? xv[1] : xv[3], 16);
-      float e = (h8 ? b : a) + __shfl_xor_sync(0xffffffffu, h8 ? a : b, 8);
-      e += __shfl_xor_sync(0xffffffffu, e, 4);
-      e += __shfl_xor_sync(0xffffffffu, e, 2);
-      e += __shfl_xor_sync(0xffffffffu, e, 1);
-      return e;
-    };
-    auto load_sz = [&](int t, float (&sc)[4], float (&zz)[4]) {
-      const int64_t ug = int64_t(tb + t) * 32 + ub + kq;
-      const uint32_t grp = units_per_group.div(uint32_t(ug < KU ? ug : 0));
-      if (rows_full && t < T && ug < KU) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          sc[i] = __half2float(srow[i * G8 + grp]);
-          zz[i] = __half2float(zrow[i * G8 + grp]);
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const bool in = t < T && ug < KU && row0 + lr + 8 * i < N;
-          sc[i] = in ? __half2float(srow[i * G8 + grp]) : 0.0f;
-          zz[i] = in ? __half2float(zrow[i * G8 + grp]) : 0.0f;
-        }
+      for (int i = 0; i < 16; ++i) {
+        const int j = tj + 8 * i;
+        if (j < gcap) tbl[trow * gcap + j] = make_float2(sv[i], zv[i]);
       }
+      asm volatile("bar.sync 1, %0;" ::"n"(32 * NW) : "memory");   // new table visible
     };
+    const uint32_t ulast = uint32_t((int64_t(te) * 32 < KU ? int64_t(te) * 32 : KU) - 1);
+    int64_t wg0 = units_per_group.div(uint32_t(tb) * 32);
+    const bool one_window = int64_t(units_per_group.div(ulast)) < wg0 + gcap;
+    load_table(wg0);
 
     uint32_t uoff[4][unit_pieces<BITS>()];
 #pragma unroll
     for (int i = 0; i < 4; ++i) unit_offsets<BITS>(lr + 8 * i, ub + kq, uoff[i]);
     float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    float xv[4], sc[4], zz[4];
-    load_x(0, xv);
-    float sx = stage_x(0, xv);
-    load_sz(0, sc, zz);
+    bool ok = true;
     for (int t = 0; t < T; ++t) {
-      float xn[4], scn[4], zzn[4];
-      load_x(t + 1, xn);
-      load_sz(t + 1, scn, zzn);
       const int s = t % D;
-      ok = mbar_wait_bounded(full0 + 8 * s, uint32_t((t / D) & 1));
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
-      __syncwarp();                      // x' of box t is visible to every lane
+      const int64_t u0 = int64_t(tb + t) * 32;         // first unit of the stage
+      if (!one_window) {
+        const int64_t ue = (u0 + 32 < KU ? u0 + 32 : KU) - 1;
+        if (int64_t(units_per_group.div(uint32_t(ue))) >= wg0 + gcap) {
+          wg0 = units_per_group.div(uint32_t(u0));
+          load_table(wg0);
+        }
+      }
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(full0 + 8 * s, uint32_t((t / D) & 1)));
+      // x' of this warp's 4 units (zero past K) and sum x of the lane's unit kq
+      const __nv_bfloat16* xr =
+          reinterpret_cast<const __nv_bfloat16*>(smem + D * Cfg::STAGE_BYTES + s * Cfg::XRAW_BYTES) +
+          ub * 32 + lane;
+      float xv[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        xv[u] = (u0 + ub + u < KU) ? __bfloat162float(xr[32 * u]) : 0.0f;
+        xs[u * XU + lane] = xv[u] * xscale;
+      }
+      float sx;
+      {
+        const bool h16 = lane & 16, h8 = lane & 8;
+        float a = (h16 ? xv[2] : xv[0]) + __shfl_xor_sync(0xffffffffu, h16 ? xv[0] : xv[2], 16);
+        float b = (h16 ? xv[3] : xv[1]) + __shfl_xor_sync(0xffffffffu, h16 ? xv[1] : xv[3], 16);
+        sx = (h8 ? b : a) + __shfl_xor_sync(0xffffffffu, h8 ? a : b, 8);
+        sx += __shfl_xor_sync(0xffffffffu, sx, 4);
+        sx += __shfl_xor_sync(0xffffffffu, sx, 2);
+        sx += __shfl_xor_sync(0xffffffffu, sx, 1);
+      }
+      __syncwarp();                      // x' is visible to every lane
       const uint32_t stage = ring + uint32_t(s * Cfg::STAGE_BYTES);
       float xp[32];
-      const float4* xq = reinterpret_cast<const float4*>(xs + (t & 1) * 128 + kq * 32);
+      const float4* xq = reinterpret_cast<const float4*>(xs + kq * XU);
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         const float4 v = xq[j];
         xp[4 * j] = v.x; xp[4 * j + 1] = v.y; xp[4 * j + 2] = v.z; xp[4 * j + 3] = v.w;
       }
+      // past K the unit's x' and sum are zero, so any table entry will do
+      int64_t grp = int64_t(units_per_group.div(uint32_t(u0 + ub + kq))) - wg0;
+      grp = grp < gcap ? grp : gcap - 1;
+      const float2* tz = tbl + lr * gcap + grp;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         uint32_t w[BITS];
@@ -356,16 +348,11 @@ gemv_m1_tma_kernel(const __grid_constant__ CUtensorMap tm_codes, const __nv_bflo
         float d[4] = {0.0f, 0.0f, 0.0f, 0.0f};
         Dot<BITS, 0>::run(w, xp, d);
         const float dot = (d[0] + d[1]) + (d[2] + d[3]);
-        acc[i] = fmaf(sc[i], fmaf(dot, 0x1p85f, -zz[i] * sx), acc[i]);
+        const float2 sz = tz[8 * i * gcap];
+        acc[i] = fmaf(sz.x, fmaf(dot, 0x1p85f, -sz.y * sx), acc[i]);
       }
-      __syncwarp();                      // this warp is done with stage s and x' buffer t & 1
+      __syncwarp();                      // this warp is done with stage s and its x' buffer
       if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(empty0 + 8 * s) : "memory");
-      sx = stage_x(t + 1, xn);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        sc[i] = scn[i];
-        zz[i] = zzn[i];
-      }
     }
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -419,14 +406,15 @@ cudaError_t launch_bits(const __nv_bfloat16* x, int64_t N, int64_t K, const uint
     return cudaErrorInvalidValue;
   static bool attr_set[64] = {};
   static int sms[64] = {};
+  constexpr int kMaxGcap = 127;
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
     cudaError_t e = cudaFuncSetAttribute(gemv_m1_tma_kernel<BITS, 2>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
-    if (e == cudaSuccess && BITS != 8)
-      e = cudaFuncSetAttribute(gemv_m1_tma_kernel<BITS, BITS == 8 ? 2 : 3>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::smem(kMaxGcap));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(gemv_m1_tma_kernel<BITS, 3>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               Cfg::smem(kMaxGcap));
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
@@ -435,15 +423,26 @@ cudaError_t launch_bits(const __nv_bfloat16* x, int64_t N, int64_t K, const uint
   // would leave SMs idle or run in a ragged second wave; every CTA keeps at
   // least WQ_GEMV_M1_MIN_STAGES stages of K so its TMA ring still pipelines.
   const int64_t tiles = (N + 31) / 32;
-  const int64_t stages = (K / 32 + 31) / 32;
+  const int64_t KU = K / 32, stages = (KU + 31) / 32;
   int ks = int((WQ_GEMV_M1_TARGET_CTAS + tiles - 1) / tiles);
   ks = ks < 1 ? 1 : (ks > 8 ? 8 : ks);
   while (ks > 1 && stages / ks < WQ_GEMV_M1_MIN_STAGES) --ks;
-  const FastDiv upg(uint32_t(g / 32));
+  // Scale table: the most groups one CTA's K range spans, odd (bank-conflict
+  // free rows), at most kMaxGcap (longer ranges reload the table).
+  const int64_t upg = g / 32;
+  int64_t span = 1;
+  for (int r = 0; r < ks; ++r) {
+    const int64_t tb = stages * r / ks, te = stages * (r + 1) / ks;
+    const int64_t ue = (te * 32 < KU ? te * 32 : KU) - 1;
+    const int64_t sp = ue / upg - (tb * 32) / upg + 1;
+    span = sp > span ? sp : span;
+  }
+  const int gcap = int(span < kMaxGcap ? span : kMaxGcap) | 1;
+  const int smem = Cfg::smem(gcap);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(unsigned(tiles), unsigned(ks), 1);
   cfg.blockDim = dim3(32 * (Cfg::NW + 1), 1, 1);
-  cfg.dynamicSmemBytes = Cfg::SMEM;
+  cfg.dynamicSmemBytes = size_t(smem);
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -452,18 +451,22 @@ cudaError_t launch_bits(const __nv_bfloat16* x, int64_t N, int64_t K, const uint
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  const FastDiv fd{uint32_t(upg)};
   // A grid between two and three CTAs per SM runs in one wave with the
-  // variant sized for three.
+  // variant sized for three, when three fit in shared memory.
   const int64_t ctas = tiles * ks, nsm = (dev >= 0 && dev < 64) ? sms[dev] : 0;
-  if (BITS != 8 && ctas > 2 * nsm && ctas <= 3 * nsm)
-    return cudaLaunchKernelEx(&cfg, gemv_m1_tma_kernel<BITS, BITS == 8 ? 2 : 3>, tm, x, N, K, scales,
-                              zeros, upg, y);
-  return cudaLaunchKernelEx(&cfg, gemv_m1_tma_kernel<BITS, 2>, tm, x, N, K, scales, zeros, upg, y);
+  if (ctas > 2 * nsm && ctas <= 3 * nsm && 3 * (smem + 1024) <= 228 * 1024)
+    return cudaLaunchKernelEx(&cfg, gemv_m1_tma_kernel<BITS, 3>, tm, x, N, K, scales, zeros, fd, gcap, y);
+  return cudaLaunchKernelEx(&cfg, gemv_m1_tma_kernel<BITS, 2>, tm, x, N, K, scales, zeros, fd, gcap, y);
 }
 
 }  // namespace
 
-bool gemv_m1_tma_supported(int64_t K, int bits) { return (K * bits) % 128 == 0; }
+bool gemv_m1_tma_supported(const void* x, const void* codes, int64_t K, int bits) {
+  // code rows and x start on 16 bytes: TMA box copies and bulk copies of x
+  return (K * bits) % 128 == 0 && (reinterpret_cast<uintptr_t>(x) & 15) == 0 &&
+         (reinterpret_cast<uintptr_t>(codes) & 15) == 0;
+}
 
 cudaError_t launch_gemv_m1_tma(const __nv_bfloat16* x, int64_t N, int64_t K,
                                const uint32_t* codes, const __half* scales, const __half* zeros,

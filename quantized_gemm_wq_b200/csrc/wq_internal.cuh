@@ -74,8 +74,9 @@ cudaError_t launch_gemv(const __nv_bfloat16* x, int M, int64_t N, int64_t K,
                         const uint32_t* codes, const __half* scales, const __half* zeros,
                         int bits, int64_t g, __nv_bfloat16* y, cudaStream_t st);
 
-// M = 1 decode GEMV with TMA-staged codes; needs 16-byte aligned code rows.
-bool gemv_m1_tma_supported(int64_t K, int bits);
+// M = 1 decode GEMV with TMA-staged codes and x; needs 16-byte aligned code
+// rows and a 16-byte aligned x.
+bool gemv_m1_tma_supported(const void* x, const void* codes, int64_t K, int bits);
 cudaError_t launch_gemv_m1_tma(const __nv_bfloat16* x, int64_t N, int64_t K,
                                const uint32_t* codes, const __half* scales, const __half* zeros,
                                int bits, int64_t g, __nv_bfloat16* y, cudaStream_t st);

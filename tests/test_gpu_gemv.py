@@ -101,3 +101,57 @@ def test_gemv_full_size_sampled(cfg, linear, M):
     oc, os_, oz = oracle_quantize(Wh[cols], bits, group)
     y_ref, bound = oracle.gemm(wq_inputs.bf16_bits(x), oc, os_, oz, len(cols), K, bits, group)
     assert_y_close(y[:, cols], y_ref, bound, f"{cfg}/{name} M={M}")
+
+
+@pytest.mark.parametrize("bits", BITS)
+@pytest.mark.parametrize("group,K", [(32, 8192), (32, 12416), (64, 16512)])
+def test_gemv_m1_long_k(bits, group, K):
+    """M = 1 over K ranges whose scale groups outnumber one shared table:
+    the table is reloaded between stages; the last stage is ragged."""
+    N = 70
+    Wh = wq_inputs.weight_f16(8, bits, N, K)
+    x = wq_inputs.activations_bf16(8, 1, 1, K)
+    y, yr, b = _run(Wh, x, bits, group)
+    assert_y_close(y, yr, b, f"bits={bits} g={group} K={K}")
+
+
+@pytest.mark.parametrize("bits", BITS)
+@pytest.mark.parametrize("offset", [1, 4, 8])
+def test_gemv_m1_offset_x(bits, offset):
+    """x starting 2, 8 or 16 bytes into a buffer: the C ABI takes 16-byte
+    aligned pointers only, so the first two are refused with status 5 and the
+    third is served."""
+    N, K, group = 70, 1280, 128
+    Wh = wq_inputs.weight_f16(9, bits, N, K)
+    x = wq_inputs.activations_bf16(9, 1, 1, K)
+    m = wq()
+    codes, s, z = m.wq_quantize_rtn(to_dev_f16(Wh), bits, group)
+    buf = torch.zeros(K + 16, dtype=torch.bfloat16, device="cuda")
+    buf[offset:offset + K] = x[0].cuda()
+    xv = buf[offset:offset + K].view(1, K)
+    if offset * 2 % 16:
+        with pytest.raises(m.WQError) as e:
+            m.wq_gemm(xv, codes, s, z, bits, group, N, K)
+        assert e.value.status == 5
+        return
+    y = m.wq_gemm(xv, codes, s, z, bits, group, N, K)
+    oc, os_, oz = oracle_quantize(Wh, bits, group)
+    y_ref, bound = oracle.gemm(wq_inputs.bf16_bits(x), oc, os_, oz, N, K, bits, group)
+    assert_y_close(y.float().cpu().numpy(), y_ref, bound, f"bits={bits} offset={offset}")
+
+
+@pytest.mark.parametrize("bits", BITS)
+def test_gemv_m1_one_hot_exact(bits):
+    """M = 1 with a one-hot x: y must equal bf16(w') of that column exactly,
+    including columns in the ragged last stage."""
+    N, K, group = 64, 1152, 64
+    Wh = wq_inputs.weight_f16(10, bits, N, K)
+    m = wq()
+    codes, s, z = m.wq_quantize_rtn(to_dev_f16(Wh), bits, group)
+    oc, os_, oz = oracle_quantize(Wh, bits, group)
+    wq_ref = oracle.dequant(oracle.unpack(oc, K, bits), os_, oz, group)
+    for k in (0, 31, 1023, 1024, 1151):
+        x = torch.zeros(1, K, dtype=torch.bfloat16)
+        x[0, k] = 1.0
+        y = m.wq_gemm(x.cuda(), codes, s, z, bits, group, N, K).cpu()
+        assert torch.equal(y[0], torch.from_numpy(wq_ref[:, k]).to(torch.bfloat16))
