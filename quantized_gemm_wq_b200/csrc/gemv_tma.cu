@@ -30,15 +30,18 @@
 // keep an absolute accuracy of 2^-64; |x| must stay below 2^63.
 #include <cuda.h>   // CUtensorMap
 
+#include "stage_smem.cuh"
 #include "wq_internal.cuh"
 
 namespace wq {
 namespace {
 
+using namespace stg;
+
 constexpr int kScaleS = 64;
 
 // The kernel is compiled for 2 resident CTAs per SM, and for 3 for grids that
-// would otherwise need a second wave of 2 per SM.
+// need fewer waves of 3 than of 2.
 // Split-K heuristic: CTAs wanted in total, and K stages kept per CTA.
 #ifndef WQ_GEMV_M1_TARGET_CTAS
 #define WQ_GEMV_M1_TARGET_CTAS 444
@@ -59,25 +62,6 @@ struct Dot {
     if constexpr (I + 1 < 32) Dot<BITS, I + 1>::run(w, xp, d);
   }
 };
-__device__ __forceinline__ uint32_t saddr(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-__device__ __forceinline__ uint64_t now_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
 __device__ __noinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
   if (mbar_try(bar, parity)) return true;
   const uint64_t t0 = now_ns();
@@ -91,28 +75,9 @@ __device__ __noinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
 }
 
 template <int BITS>
-__device__ __forceinline__ void lds_words(uint32_t a, uint32_t (&w)[BITS]) {
-  if constexpr (BITS == 2) {
-    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(w[0]), "=r"(w[1]) : "r"(a));
-  } else if constexpr (BITS == 4) {
-    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]) : "r"(a));
-  } else if constexpr (BITS == 8) {
-    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]) : "r"(a));
-    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(w[4]), "=r"(w[5]), "=r"(w[6]), "=r"(w[7]) : "r"(a + 16));
-  } else {
-    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(w[0]) : "r"(a));
-    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(w[1]) : "r"(a + 4));
-    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(w[2]) : "r"(a + 8));
-  }
-}
-
-template <int BITS>
 struct M1Cfg {
   static constexpr int NW = 8;                       // consumer warps (4 units of a stage each)
-  static constexpr int D = BITS == 8 ? 3 : 4;        // ring stages
+  static constexpr int D = 3;                        // ring stages
   static constexpr int STAGE_WORDS = 32 * BITS;      // 32 units of one row
   static constexpr int BOX_BYTES = 32 * 128;         // one TMA box: 32 rows x 128 bytes, swizzled
   static constexpr int STAGE_BYTES = BITS * BOX_BYTES;
@@ -123,54 +88,6 @@ struct M1Cfg {
   static constexpr int FIXED = D * (STAGE_BYTES + XRAW_BYTES) + XS_BYTES + 2 * D * 8;
   static int smem(int gcap) { return FIXED + 32 * gcap * 8 + 1024; }
 };
-
-// Shared-memory byte offset of word wi (0 .. 32*BITS-1) of row r in a stage:
-// the stage holds BITS boxes of 32 words per row; inside a box, rows are 128
-// bytes apart and the 16-byte chunk index is XOR-ed with r % 8 (128B swizzle).
-__device__ __forceinline__ uint32_t swz_word(int r, int wi) {
-  const int box = wi >> 5, c = (wi >> 2) & 7, e = wi & 3;
-  return uint32_t(box * 4096 + r * 128 + ((c ^ (r & 7)) << 4) + (e << 2));
-}
-
-// Shared-memory offsets of the pieces of unit u of row r in a stage: one
-// vector per 16-byte chunk (b = 2, 4, 8: 1, 1, 2 pieces) or one per word
-// (b = 3: 3 pieces).  They do not depend on the stage, so each lane computes
-// them once.
-template <int BITS>
-constexpr int unit_pieces() { return BITS == 3 ? 3 : (BITS == 8 ? 2 : 1); }
-
-template <int BITS>
-__device__ __forceinline__ void unit_offsets(int r, int u, uint32_t (&o)[unit_pieces<BITS>()]) {
-  if constexpr (BITS == 3) {
-#pragma unroll
-    for (int j = 0; j < 3; ++j) o[j] = swz_word(r, 3 * u + j);
-  } else if constexpr (BITS == 8) {
-    o[0] = swz_word(r, 8 * u);
-    o[1] = swz_word(r, 8 * u + 4);
-  } else {
-    o[0] = swz_word(r, BITS * u);
-  }
-}
-
-template <int BITS>
-__device__ __forceinline__ void load_unit_at(uint32_t stage, const uint32_t (&o)[unit_pieces<BITS>()],
-                                             uint32_t (&w)[BITS]) {
-  if constexpr (BITS == 4) {
-    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]) : "r"(stage + o[0]));
-  } else if constexpr (BITS == 2) {
-    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(w[0]), "=r"(w[1]) : "r"(stage + o[0]));
-  } else if constexpr (BITS == 8) {
-    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]) : "r"(stage + o[0]));
-    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(w[4]), "=r"(w[5]), "=r"(w[6]), "=r"(w[7]) : "r"(stage + o[1]));
-  } else {
-#pragma unroll
-    for (int j = 0; j < 3; ++j)
-      asm volatile("ld.shared.u32 %0, [%1];" : "=r"(w[j]) : "r"(stage + o[j]));
-  }
-}
 
 // One CTA: 32 output rows over its share of K.  Warp NW is the producer: one
 // lane issues, per stage, the TMA copy of the 32-row x 32-unit box of codes and
@@ -452,10 +369,10 @@ cudaError_t launch_bits(const __nv_bfloat16* x, int64_t N, int64_t K, const uint
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   const FastDiv fd{uint32_t(upg)};
-  // A grid between two and three CTAs per SM runs in one wave with the
-  // variant sized for three, when three fit in shared memory.
-  const int64_t ctas = tiles * ks, nsm = (dev >= 0 && dev < 64) ? sms[dev] : 0;
-  if (ctas > 2 * nsm && ctas <= 3 * nsm && 3 * (smem + 1024) <= 228 * 1024)
+  // The variant sized for three CTAs per SM, when three fit in shared memory
+  // and the grid then runs in fewer waves.
+  const int64_t ctas = tiles * ks, nsm = (dev >= 0 && dev < 64 && sms[dev] > 0) ? sms[dev] : 1;
+  if ((ctas + 3 * nsm - 1) / (3 * nsm) < (ctas + 2 * nsm - 1) / (2 * nsm) && 3 * (smem + 1024) <= 228 * 1024)
     return cudaLaunchKernelEx(&cfg, gemv_m1_tma_kernel<BITS, 3>, tm, x, N, K, scales, zeros, fd, gcap, y);
   return cudaLaunchKernelEx(&cfg, gemv_m1_tma_kernel<BITS, 2>, tm, x, N, K, scales, zeros, fd, gcap, y);
 }

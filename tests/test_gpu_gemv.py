@@ -155,3 +155,48 @@ def test_gemv_m1_one_hot_exact(bits):
         x[0, k] = 1.0
         y = m.wq_gemm(x.cuda(), codes, s, z, bits, group, N, K).cpu()
         assert torch.equal(y[0], torch.from_numpy(wq_ref[:, k]).to(torch.bfloat16))
+
+
+@pytest.mark.parametrize("bits", BITS)
+@pytest.mark.parametrize("N,K,group", [(70, 1152, 128), (70, 1152, 384), (33, 2048, 0), (100, 5120, 256),
+                                       (40, 128, 128)])
+def test_gemv_m1_tma_groups(bits, N, K, group):
+    """M = 1 with K a multiple of 128 (TMA-staged codes): ragged N, a 128-code
+    last stage at K = 1152, groups of 128, 256 and 384 and a per-row grid."""
+    Wh = wq_inputs.weight_f16(11, bits, N, K, dist="t4")
+    x = wq_inputs.activations_bf16(11, 1, 1, K)
+    y, yr, b = _run(Wh, x, bits, group)
+    assert_y_close(y, yr, b, f"bits={bits} N={N} K={K} g={group}")
+
+
+@pytest.mark.parametrize("bits", BITS)
+def test_gemv_m1_one_hot_exact_g128(bits):
+    """M = 1, g = 128, one nonzero x: a single exact product per row, so
+    y = bf16(-3 w') exactly."""
+    N, K, group = 64, 1152, 128
+    Wh = wq_inputs.weight_f16(12, bits, N, K)
+    m = wq()
+    codes, s, z = m.wq_quantize_rtn(to_dev_f16(Wh), bits, group)
+    oc, os_, oz = oracle_quantize(Wh, bits, group)
+    wq_ref = oracle.dequant(oracle.unpack(oc, K, bits), os_, oz, group)
+    for k in (0, 5, 31, 127, 128, 1023, 1024, 1151):
+        x = torch.zeros(1, K, dtype=torch.bfloat16)
+        x[0, k] = -3.0
+        y = m.wq_gemm(x.cuda(), codes, s, z, bits, group, N, K).cpu()
+        assert torch.equal(y[0], (-3.0 * torch.from_numpy(wq_ref[:, k])).to(torch.bfloat16)), k
+
+
+def test_gemv_m1_table_windows_g128():
+    """N = 14240, K = 16512, g = 128: one CTA's K range spans 129 groups, more
+    than its scale table holds, so the table is reloaded between stages;
+    checked on sampled rows."""
+    N, K, bits, group = 14240, 16512, 2, 128
+    Wh = wq_inputs.weight_f16(13, bits, N, K)
+    x = wq_inputs.activations_bf16(13, 1, 1, K)
+    m = wq()
+    codes, s, z = m.wq_quantize_rtn(to_dev_f16(Wh), bits, group)
+    y = m.wq_gemm(x.cuda(), codes, s, z, bits, group, N, K).float().cpu().numpy()
+    cols = np.unique(np.concatenate([[0, N - 1], np.random.default_rng(9).integers(0, N, 126)]))
+    oc, os_, oz = oracle_quantize(Wh[cols], bits, group)
+    y_ref, bound = oracle.gemm(wq_inputs.bf16_bits(x), oc, os_, oz, len(cols), K, bits, group)
+    assert_y_close(y[:, cols], y_ref, bound, "table windows")
