@@ -146,6 +146,9 @@ gemv_m1_tma_kernel(const __grid_constant__ CUtensorMap tm_codes, const __nv_bflo
       for (int t = 0; t < T && ok; ++t) {
         const int s = t % D;
         if (t >= D) ok = mbar_wait_bounded(empty0 + 8 * s, uint32_t(((t / D) - 1) & 1));
+        // the first stage goes out alone: with every CTA's whole ring in flight at once
+        // the memory system returns the first stages late
+        if (t == 1) ok = ok && mbar_wait_bounded(full0, 0u);
         if (!ok) break;
         const int64_t k0 = int64_t(tb + t) * 1024;
         const uint32_t xbytes = uint32_t((K - k0 < 1024 ? K - k0 : 1024) * 2);
