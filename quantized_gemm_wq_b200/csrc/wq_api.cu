@@ -119,7 +119,9 @@ wq_status wq_gemm(const void* x_bf16, int64_t M, int64_t N, int64_t K, const uin
     e = cudaSuccess;
     for (int64_t m0 = 0; m0 < M && e == cudaSuccess; m0 += wq::kGemvMaxM) {
       const int mc = int(M - m0 < wq::kGemvMaxM ? M - m0 : wq::kGemvMaxM);
-      if (wq::gemv_tc_supported(mc, K, bits, g))
+      if (wq::gemv_mma_supported(mc, x + m0 * K, codes, K, g))
+        e = wq::launch_gemv_mma(x + m0 * K, mc, N, K, codes, s, z, bits, g, y + m0 * N, strm);
+      else if (wq::gemv_tc_supported(mc, K, bits, g))
         e = wq::launch_gemv_tc(x + m0 * K, mc, N, K, codes, s, z, bits, g, y + m0 * N, strm);
       else
         e = wq::launch_gemv(x + m0 * K, mc, N, K, codes, s, z, bits, g, y + m0 * N, strm);
@@ -129,12 +131,13 @@ wq_status wq_gemm(const void* x_bf16, int64_t M, int64_t N, int64_t K, const uin
 }
 
 wq_status wq_last_device_error(void) {
-  cudaError_t e1 = cudaSuccess, e2 = cudaSuccess, e3 = cudaSuccess;
+  cudaError_t e1 = cudaSuccess, e2 = cudaSuccess, e3 = cudaSuccess, e4 = cudaSuccess;
   const bool hit1 = wq::gemm_tc_read_and_clear_timeout(&e1);
   const bool hit2 = wq::gemv_m1_tma_read_and_clear_timeout(&e2);
   const bool hit3 = wq::gemv_tc_read_and_clear_timeout(&e3);
-  if (e1 != cudaSuccess || e2 != cudaSuccess || e3 != cudaSuccess) return WQ_ERR_CUDA;
-  return (hit1 || hit2 || hit3) ? WQ_ERR_DEVICE_TIMEOUT : WQ_OK;
+  const bool hit4 = wq::gemv_mma_read_and_clear_timeout(&e4);
+  if (e1 != cudaSuccess || e2 != cudaSuccess || e3 != cudaSuccess || e4 != cudaSuccess) return WQ_ERR_CUDA;
+  return (hit1 || hit2 || hit3 || hit4) ? WQ_ERR_DEVICE_TIMEOUT : WQ_OK;
 }
 
 }  // extern "C"

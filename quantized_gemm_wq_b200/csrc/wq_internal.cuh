@@ -82,6 +82,14 @@ cudaError_t launch_gemv_m1_tma(const __nv_bfloat16* x, int64_t N, int64_t K,
                                int bits, int64_t g, __nv_bfloat16* y, cudaStream_t st);
 bool gemv_m1_tma_read_and_clear_timeout(cudaError_t* err);
 
+// Decode GEMV for 2..8 tokens on warp-level MMAs (gemv_mma.cu): K and the group
+// length multiples of 128, x rows and code rows 16-byte aligned.
+bool gemv_mma_supported(int M, const void* x, const void* codes, int64_t K, int64_t g);
+cudaError_t launch_gemv_mma(const __nv_bfloat16* x, int M, int64_t N, int64_t K, const uint32_t* codes,
+                            const __half* scales, const __half* zeros, int bits, int64_t g,
+                            __nv_bfloat16* y, cudaStream_t st);
+bool gemv_mma_read_and_clear_timeout(cudaError_t* err);
+
 // True when the tensor-core path can stage this K with TMA (K a multiple of 128).
 bool gemm_tc_supported(int64_t K, int bits);
 

@@ -200,3 +200,37 @@ def test_gemv_m1_table_windows_g128():
     oc, os_, oz = oracle_quantize(Wh[cols], bits, group)
     y_ref, bound = oracle.gemm(wq_inputs.bf16_bits(x), oc, os_, oz, len(cols), K, bits, group)
     assert_y_close(y[:, cols], y_ref, bound, "table windows")
+
+
+@pytest.mark.parametrize("bits", BITS)
+@pytest.mark.parametrize("M", [2, 3, 6, 8])
+@pytest.mark.parametrize("N,K,group", [(70, 1152, 128), (33, 2048, 0), (100, 1280, 256)])
+def test_gemv_small_batch_quads(bits, M, N, K, group):
+    """2..8 tokens with K and the group length in whole 128-code quads (the
+    warp-level MMA GEMV): ragged N, a one-quad last stage, per-row grids."""
+    Wh = wq_inputs.weight_f16(14, bits, N, K, dist="t4")
+    x = wq_inputs.activations_bf16(14, M, M, K)
+    y, yr, b = _run(Wh, x, bits, group)
+    assert_y_close(y, yr, b, f"bits={bits} M={M} N={N} K={K} g={group}")
+
+
+@pytest.mark.parametrize("bits", BITS)
+@pytest.mark.parametrize("M", [2, 5, 8])
+def test_gemv_small_batch_one_hot_exact_g128(bits, M):
+    """2..8 tokens, g = 128: token m is one-hot at column k_m (one exact
+    product per output), the last token is all zero."""
+    N, K, group = 64, 1152, 128
+    Wh = wq_inputs.weight_f16(15, bits, N, K)
+    m = wq()
+    codes, s, z = m.wq_quantize_rtn(to_dev_f16(Wh), bits, group)
+    oc, os_, oz = oracle_quantize(Wh, bits, group)
+    wq_ref = oracle.dequant(oracle.unpack(oc, K, bits), os_, oz, group)
+    ks = [0, 31, 127, 128, 1023, 1024, 1151, 600][:M - 1]
+    x = torch.zeros(M, K, dtype=torch.bfloat16)
+    for i, k in enumerate(ks):
+        x[i, k] = 2.0 if i % 2 else -1.0
+    y = m.wq_gemm(x.cuda(), codes, s, z, bits, group, N, K).cpu()
+    for i, k in enumerate(ks):
+        ref = ((2.0 if i % 2 else -1.0) * torch.from_numpy(wq_ref[:, k])).to(torch.bfloat16)
+        assert torch.equal(y[i], ref), (i, k)
+    assert torch.equal(y[M - 1], torch.zeros(N, dtype=torch.bfloat16))

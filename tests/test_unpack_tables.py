@@ -1,7 +1,8 @@
-"""The tensor-core GEMV's unpack tables (host data of the CUDA path, checked on
+"""The tensor-core GEMVs' unpack tables (host data of the CUDA path, checked on
 the CPU): every AND of a table must pull exactly the codes it names out of a
-segment packed by the oracle's packer, each code once, in the low byte of its
-16-bit half (where bf16 bit patterns are linear in value)."""
+128-code segment (kUnpack) or a 32-code unit (kUnit) packed by the oracle's
+packer, each code once, in the low byte of its 16-bit half (where bf16 bit
+patterns are linear in value)."""
 import os
 import re
 
@@ -14,10 +15,10 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "quantized_gemm_wq_b200", "csrc", "unpack_tables.h")
 
 
-def parse_tables():
+def parse_tables(family="kUnpack", n=64):
     text = open(HEADER).read()
     out = {}
-    for bits, body in re.findall(r"kUnpack(\d)\[64\] = \{(.*?)\};", text, re.S):
+    for bits, body in re.findall(family + r"(\d)\[" + str(n) + r"\] = \{(.*?)\};", text, re.S):
         ops = re.findall(r"\{(\d+), 0x([0-9A-F]+)u, (\d+), (\d+), (\d+), (\d+)\}", body)
         out[int(bits)] = [(int(s), int(m, 16), int(a), int(b), int(c), int(d)) for s, m, a, b, c, d in ops]
     return out
@@ -32,15 +33,16 @@ def test_header_is_generated():
     assert open(HEADER).read() == gen.render()
 
 
+@pytest.mark.parametrize("family,nc", [("kUnpack", 128), ("kUnit", 32)])
 @pytest.mark.parametrize("bits", [2, 3, 4, 8])
-def test_ops_extract_each_code_once(bits):
-    ops = parse_tables()[bits]
-    assert len(ops) == 64
+def test_ops_extract_each_code_once(bits, family, nc):
+    ops = parse_tables(family, nc // 2)[bits]
+    assert len(ops) == nc // 2
     seen = sorted([o[2] for o in ops] + [o[4] for o in ops])
-    assert seen == list(range(128))
+    assert seen == list(range(nc))
     rng = np.random.default_rng(bits)
     for trial in range(20):
-        q = rng.integers(0, 1 << bits, size=(1, 128), dtype=np.uint8)
+        q = rng.integers(0, 1 << bits, size=(1, nc), dtype=np.uint8)
         if trial == 0:
             q[:] = (1 << bits) - 1                      # all bits set: masks must not leak
         words = oracle.pack(q, bits)[0]
@@ -69,3 +71,6 @@ def test_shift_counts():
     shifts = {b: len({o[0] for o in ops if o[0] % 32}) for b, ops in t.items()}
     assert shifts[2] == 8 and shifts[4] == 16 and shifts[8] == 32
     assert shifts[3] <= 28
+    u = parse_tables("kUnit", 16)
+    ushifts = {b: len({o[0] for o in ops if o[0] % 32}) for b, ops in u.items()}
+    assert ushifts[2] == 2 and ushifts[4] == 4 and ushifts[8] == 8 and ushifts[3] <= 7
