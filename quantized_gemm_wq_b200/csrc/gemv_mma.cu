@@ -141,6 +141,31 @@ struct TileMma {
   }
 };
 
+// Sums of MT per-token values over the warp, one token per lane: at each step
+// lanes keep half of their tokens and add the partner's copy of that half, so
+// after log2(MT) steps lane l holds a partial of token (l >> (5 - log2 MT)),
+// completed by the remaining xor steps.  MT - 1 + 5 - log2(MT) shuffles
+// instead of 5 MT.
+template <int MT>
+__device__ __forceinline__ float token_sums(float (&p)[MT], int lane) {
+  constexpr int LG = MT == 2 ? 1 : (MT == 4 ? 2 : 3);
+  static_assert(MT == (1 << LG), "MT must be 2, 4 or 8");
+#pragma unroll
+  for (int step = 0; step < LG; ++step) {
+    const int d = 16 >> step, half = MT >> (step + 1);
+    const bool hi = lane & d;
+#pragma unroll
+    for (int i = 0; i < half; ++i) {
+      const float keep = hi ? p[half + i] : p[i], send = hi ? p[i] : p[half + i];
+      p[i] = keep + __shfl_xor_sync(0xffffffffu, send, d);
+    }
+  }
+  float r = p[0];
+#pragma unroll
+  for (int d = 16 >> LG; d >= 1; d >>= 1) r += __shfl_xor_sync(0xffffffffu, r, d);
+  return r;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
@@ -268,19 +293,16 @@ gemv_mma_kernel(const __grid_constant__ CUtensorMap tm_codes, const __nv_bfloat1
     // acc[r][c]: row g + 8 r, token 2 tq + c
     float acc[4][2] = {};
     float c0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, c1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    float sxg[MT];                               // sum x of the group so far, per token
-#pragma unroll
-    for (int m = 0; m < MT; ++m) sxg[m] = 0.0f;
+    // sum x of the group so far, of token lane >> (5 - log2 MT) (see token_sums)
+    constexpr int kTokShift = MT == 2 ? 4 : (MT == 4 ? 3 : 2);
+    float sxg = 0.0f;
     int64_t cur = -1;                            // group of the accumulators
     auto flush = [&]() {
       int64_t gi = cur - wg0;
       gi = gi < gcap ? gi : gcap - 1;
-      float s0 = 0.0f, s1 = 0.0f;                // sum x of tokens 2 tq and 2 tq + 1
-#pragma unroll
-      for (int m = 0; m < MT; ++m) {
-        s0 = (m == 2 * tq) ? sxg[m] : s0;
-        s1 = (m == 2 * tq + 1) ? sxg[m] : s1;
-      }
+      // sum x of tokens 2 tq and 2 tq + 1 (a token past MT reads some lane: unused)
+      const float s0 = __shfl_sync(0xffffffffu, sxg, ((2 * tq) << kTokShift) & 31);
+      const float s1 = __shfl_sync(0xffffffffu, sxg, ((2 * tq + 1) << kTokShift) & 31);
       const float2 sz[4] = {tbl[g * gcap + gi], tbl[(g + 8) * gcap + gi], tbl[(g + 16) * gcap + gi],
                             tbl[(g + 24) * gcap + gi]};
       const float cc[4][2] = {{c0[0], c0[1]}, {c0[2], c0[3]}, {c1[0], c1[1]}, {c1[2], c1[3]}};
@@ -291,8 +313,7 @@ gemv_mma_kernel(const __grid_constant__ CUtensorMap tm_codes, const __nv_bfloat1
       }
 #pragma unroll
       for (int i = 0; i < 4; ++i) c0[i] = c1[i] = 0.0f;
-#pragma unroll
-      for (int m = 0; m < MT; ++m) sxg[m] = 0.0f;
+      sxg = 0.0f;
     };
     bool ok = true;
     for (int t = 0; t < T; ++t) {
@@ -312,6 +333,7 @@ gemv_mma_kernel(const __grid_constant__ CUtensorMap tm_codes, const __nv_bfloat1
       if (ok) ok = __all_sync(0xffffffffu, mma_wait_bounded(full0 + 8 * s, uint32_t((t / D) & 1)));
       // x' of the quad for every token: this lane's two words, and sum x over the quad
       const bool uin = q0 + xu < KU;
+      float px[MT];
 #pragma unroll
       for (int m = 0; m < MT; ++m) {
         const __nv_bfloat16* xr =
@@ -322,14 +344,9 @@ gemv_mma_kernel(const __grid_constant__ CUtensorMap tm_codes, const __nv_bfloat1
         const float xl1 = in ? __bfloat162float(xr[lo1]) : 0.0f, xh1 = in ? __bfloat162float(xr[hi1]) : 0.0f;
         *reinterpret_cast<uint2*>(xpw + (m * 4 + xu) * XB + xpair) =
             make_uint2(pack_bf16x2(xl0 * flo0, xh0 * fhi0), pack_bf16x2(xl1 * flo1, xh1 * fhi1));
-        float sx = (xl0 + xh0) + (xl1 + xh1);
-        sx += __shfl_xor_sync(0xffffffffu, sx, 16);
-        sx += __shfl_xor_sync(0xffffffffu, sx, 8);
-        sx += __shfl_xor_sync(0xffffffffu, sx, 4);
-        sx += __shfl_xor_sync(0xffffffffu, sx, 2);
-        sx += __shfl_xor_sync(0xffffffffu, sx, 1);
-        sxg[m] += sx;
+        px[m] = (xl0 + xh0) + (xl1 + xh1);
       }
+      sxg += token_sums<MT>(px, lane);
       __syncwarp();                                     // x' visible to the warp
       uint32_t xb[16];
 #pragma unroll
