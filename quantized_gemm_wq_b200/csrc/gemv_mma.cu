@@ -330,7 +330,10 @@ gemv_mma_kernel(const __grid_constant__ CUtensorMap tm_codes, const __nv_bfloat1
         }
       }
       cur = grp;
-      if (ok) ok = __all_sync(0xffffffffu, mma_wait_bounded(full0 + 8 * s, uint32_t((t / D) & 1)));
+      {   // the common case (stage landed) without the call to the bounded wait
+        const uint32_t par = uint32_t((t / D) & 1);
+        if (ok) ok = __all_sync(0xffffffffu, mbar_try(full0 + 8 * s, par) || mma_wait_bounded(full0 + 8 * s, par));
+      }
       // x' of the quad for every token: this lane's two words, and sum x over the quad
       const bool uin = q0 + xu < KU;
       float px[MT];

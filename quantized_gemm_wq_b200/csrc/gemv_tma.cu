@@ -227,7 +227,10 @@ gemv_m1_tma_kernel(const __grid_constant__ CUtensorMap tm_codes, const __nv_bflo
           load_table(wg0);
         }
       }
-      if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(full0 + 8 * s, uint32_t((t / D) & 1)));
+      {   // the common case (stage landed) without the call to the bounded wait
+        const uint32_t par = uint32_t((t / D) & 1);
+        if (ok) ok = __all_sync(0xffffffffu, mbar_try(full0 + 8 * s, par) || mbar_wait_bounded(full0 + 8 * s, par));
+      }
       // x' of this warp's 4 units (zero past K) and sum x of the lane's unit kq
       const __nv_bfloat16* xr =
           reinterpret_cast<const __nv_bfloat16*>(smem + D * Cfg::STAGE_BYTES + s * Cfg::XRAW_BYTES) +
