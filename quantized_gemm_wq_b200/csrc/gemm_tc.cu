@@ -30,6 +30,8 @@
 // stop, drain its copies in flight and free its tensor memory.
 #include <cuda.h>   // CUtensorMap types only; the driver entry point is fetched at run time
 
+#include <atomic>
+
 #include "wq_internal.cuh"
 
 namespace wq {
@@ -580,11 +582,12 @@ constexpr double kSplitStages = 3.0;   // partial-tile exchange per extra split
 // per device and cluster size.  0 if the query fails.
 template <int BITS>
 int cluster_slots(int dev, int c, uint32_t smem) {
-  static int cache[64][4] = {};
+  static std::atomic<int> cache[64][4];   // 0 unknown, -1 query failed
   int ci = 0;
   while ((1 << ci) < c) ++ci;
   if (dev < 0 || dev >= 64 || ci > 3) return 0;
-  if (cache[dev][ci] != 0) return cache[dev][ci] > 0 ? cache[dev][ci] : 0;
+  const int known = cache[dev][ci].load(std::memory_order_relaxed);
+  if (known != 0) return known > 0 ? known : 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(1, 1, unsigned(c));
   cfg.blockDim = dim3(kThreads, 1, 1);
@@ -599,10 +602,10 @@ int cluster_slots(int dev, int c, uint32_t smem) {
   int n = 0;
   if (cudaOccupancyMaxActiveClusters(&n, gemm_tc_kernel<BITS>, &cfg) != cudaSuccess || n <= 0) {
     cudaGetLastError();
-    cache[dev][ci] = -1;
+    cache[dev][ci].store(-1, std::memory_order_relaxed);
     return 0;
   }
-  cache[dev][ci] = n;
+  cache[dev][ci].store(n, std::memory_order_relaxed);
   return n;
 }
 
@@ -617,14 +620,15 @@ cudaError_t launch_bits(const __nv_bfloat16* x, int64_t M, int64_t N, int64_t K,
                           uint64_t(K * BITS / 8), CK * BITS / 32, BN, 0))
     return cudaErrorInvalidValue;
   constexpr uint32_t smem = TcCfg<BITS>::kSmem;
-  static bool attr_set[64] = {};
+  // per device, set once; concurrent first calls repeat an idempotent call
+  static std::atomic<bool> attr_set[64];
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+  if (dev >= 0 && dev < 64 && !attr_set[dev].load(std::memory_order_acquire)) {
     cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BITS>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
     if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
+    attr_set[dev].store(true, std::memory_order_release);
   }
   // Split K over a cluster when the output tiles alone fill the SMs badly.
   // Cost model in units of one 128-wide code stage: every wave of clusters

@@ -35,6 +35,8 @@
 // across a split-K cluster through distributed shared memory.
 #include <cuda.h>   // CUtensorMap
 
+#include <atomic>
+
 #include "stage_smem.cuh"
 #include "unpack_tables.h"
 #include "wq_internal.cuh"
@@ -425,20 +427,23 @@ cudaError_t launch_mt(const __nv_bfloat16* x, int M, int64_t N, int64_t K, const
   if (!make_tensor_map_2d(&tm, TmaType::kU32, codes, uint64_t(K * BITS / 32), uint64_t(N),
                           uint64_t(K * BITS / 8), 32, 32, 128))
     return cudaErrorInvalidValue;
-  static bool attr_set[64] = {};
-  static int sms[64] = {};
+  // per device, set once; concurrent first calls repeat idempotent queries
+  static std::atomic<bool> attr_set[64];
+  static std::atomic<int> sms[64];
   constexpr int kMaxGcap = 127;
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+  if (dev >= 0 && dev < 64 && !attr_set[dev].load(std::memory_order_acquire)) {
     cudaError_t e = cudaFuncSetAttribute(gemv_mma_kernel<BITS, MT, 2>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::smem(kMaxGcap));
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(gemv_mma_kernel<BITS, MT, 3>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                Cfg::smem(kMaxGcap));
-    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev);
+    int nsm_dev = 0;
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&nsm_dev, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
+    sms[dev].store(nsm_dev, std::memory_order_relaxed);
+    attr_set[dev].store(true, std::memory_order_release);
   }
   const int64_t tiles = (N + 31) / 32;
   const int64_t KU = K / 32, stages = (KU + 31) / 32;
@@ -468,7 +473,8 @@ cudaError_t launch_mt(const __nv_bfloat16* x, int M, int64_t N, int64_t K, const
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   const FastDiv fd{uint32_t(upg)};
-  const int64_t ctas = tiles * ks, nsm = (dev >= 0 && dev < 64 && sms[dev] > 0) ? sms[dev] : 1;
+  const int nsm_known = (dev >= 0 && dev < 64) ? sms[dev].load(std::memory_order_relaxed) : 0;
+  const int64_t ctas = tiles * ks, nsm = nsm_known > 0 ? nsm_known : 1;
   constexpr int kRed = int(sizeof(float)) * Cfg::NW * MT * 32;   // static shared memory
   if ((ctas + 3 * nsm - 1) / (3 * nsm) < (ctas + 2 * nsm - 1) / (2 * nsm) &&
       3 * (smem + kRed + 1024) <= 228 * 1024)

@@ -43,6 +43,7 @@
 // read by wq_last_device_error, and the CTA drains and leaves.
 #include <cuda.h>
 
+#include <atomic>
 #include <algorithm>
 
 #include "tc_unpack.cuh"
@@ -455,9 +456,10 @@ constexpr double kSplitSegs = 1.0;     // cluster reduction
 
 template <int BITS, int MP>
 int cluster_slots(int dev, int c, uint32_t smem) {
-  static int cache[64][kMaxSplit + 1] = {};
+  static std::atomic<int> cache[64][kMaxSplit + 1];   // 0 unknown, -1 query failed
   if (dev < 0 || dev >= 64 || c < 1 || c > kMaxSplit) return 0;
-  if (cache[dev][c] != 0) return cache[dev][c] > 0 ? cache[dev][c] : 0;
+  const int known = cache[dev][c].load(std::memory_order_relaxed);
+  if (known != 0) return known > 0 ? known : 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(1, unsigned(c), 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
@@ -472,10 +474,10 @@ int cluster_slots(int dev, int c, uint32_t smem) {
   int n = 0;
   if (cudaOccupancyMaxActiveClusters(&n, gemv_tc_kernel<BITS, MP>, &cfg) != cudaSuccess || n <= 0) {
     cudaGetLastError();
-    cache[dev][c] = -1;
+    cache[dev][c].store(-1, std::memory_order_relaxed);
     return 0;
   }
-  cache[dev][c] = n;
+  cache[dev][c].store(n, std::memory_order_relaxed);
   return n;
 }
 
@@ -516,14 +518,15 @@ cudaError_t launch_tc(const __nv_bfloat16* x, int M, int64_t N, int64_t K, const
                           uint64_t(K * BITS / 8), uint32_t(C::kWords), kRows, C::kSwzBytes))
     return cudaErrorInvalidValue;
   constexpr uint32_t smem = TcvSmem<BITS, MP>::kTotal;
-  static bool attr_set[64] = {};
+  // per device, set once; concurrent first calls repeat an idempotent call
+  static std::atomic<bool> attr_set[64];
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+  if (dev >= 0 && dev < 64 && !attr_set[dev].load(std::memory_order_acquire)) {
     cudaError_t e = cudaFuncSetAttribute(gemv_tc_kernel<BITS, MP>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
     if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
+    attr_set[dev].store(true, std::memory_order_release);
   }
   const int nseg = int(K / kSeg);
   const int64_t tiles = (N + kRows - 1) / kRows;

@@ -30,6 +30,8 @@
 // keep an absolute accuracy of 2^-64; |x| must stay below 2^63.
 #include <cuda.h>   // CUtensorMap
 
+#include <atomic>
+
 #include "stage_smem.cuh"
 #include "wq_internal.cuh"
 
@@ -327,20 +329,23 @@ cudaError_t launch_bits(const __nv_bfloat16* x, int64_t N, int64_t K, const uint
   if (!make_tensor_map_2d(&tm, TmaType::kU32, codes, uint64_t(K * BITS / 32), uint64_t(N),
                           uint64_t(K * BITS / 8), 32, 32, 128))
     return cudaErrorInvalidValue;
-  static bool attr_set[64] = {};
-  static int sms[64] = {};
+  // per device, set once; concurrent first calls repeat idempotent queries
+  static std::atomic<bool> attr_set[64];
+  static std::atomic<int> sms[64];
   constexpr int kMaxGcap = 127;
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+  if (dev >= 0 && dev < 64 && !attr_set[dev].load(std::memory_order_acquire)) {
     cudaError_t e = cudaFuncSetAttribute(gemv_m1_tma_kernel<BITS, 2>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::smem(kMaxGcap));
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(gemv_m1_tma_kernel<BITS, 3>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                Cfg::smem(kMaxGcap));
-    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev);
+    int nsm_dev = 0;
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&nsm_dev, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
+    sms[dev].store(nsm_dev, std::memory_order_relaxed);
+    attr_set[dev].store(true, std::memory_order_release);
   }
   // Split K over a cluster of ks CTAs (at most 8) when the row tiles alone
   // would leave SMs idle or run in a ragged second wave; every CTA keeps at
@@ -377,7 +382,8 @@ cudaError_t launch_bits(const __nv_bfloat16* x, int64_t N, int64_t K, const uint
   const FastDiv fd{uint32_t(upg)};
   // The variant sized for three CTAs per SM, when three fit in shared memory
   // and the grid then runs in fewer waves.
-  const int64_t ctas = tiles * ks, nsm = (dev >= 0 && dev < 64 && sms[dev] > 0) ? sms[dev] : 1;
+  const int nsm_known = (dev >= 0 && dev < 64) ? sms[dev].load(std::memory_order_relaxed) : 0;
+  const int64_t ctas = tiles * ks, nsm = nsm_known > 0 ? nsm_known : 1;
   if ((ctas + 3 * nsm - 1) / (3 * nsm) < (ctas + 2 * nsm - 1) / (2 * nsm) && 3 * (smem + 1024) <= 228 * 1024)
     return cudaLaunchKernelEx(&cfg, gemv_m1_tma_kernel<BITS, 3>, tm, x, N, K, scales, zeros, fd, gcap, y);
   return cudaLaunchKernelEx(&cfg, gemv_m1_tma_kernel<BITS, 2>, tm, x, N, K, scales, zeros, fd, gcap, y);
