@@ -74,3 +74,22 @@ def test_shift_counts():
     u = parse_tables("kUnit", 16)
     ushifts = {b: len({o[0] for o in ops if o[0] % 32}) for b, ops in u.items()}
     assert ushifts[2] == 2 and ushifts[4] == 4 and ushifts[8] == 8 and ushifts[3] <= 7
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+def test_unit_products_share_one_scale(bits):
+    """For every AND of the 32-code unit table: the bf16 pattern of code q at
+    offset b times bf16(x 2^(64 - b)) is q x 2^-69 exactly, for every code and
+    sampled bf16 activations (the warp-MMA GEMV sums these products in fp32)."""
+    ops = parse_tables("kUnit", 16)[bits]
+    rng = np.random.default_rng(100 + bits)
+    xs = (rng.standard_normal(64) * np.exp2(rng.integers(-20, 20, 64))).astype(np.float32)
+    xs = (xs.view(np.uint32) & 0xFFFF0000).view(np.float32)          # bf16-representable
+    for s, m, lo, blo, hi, bhi in ops:
+        for b in (blo, bhi):
+            for q in range(1 << bits):
+                a = np.array([(q << b) << 16], dtype=np.uint32).view(np.float32)[0]
+                xp = (xs.astype(np.float64) * 2.0 ** (64 - b)).astype(np.float32)
+                assert np.all((xp.view(np.uint32) & 0xFFFF) == 0)     # still bf16: scaling is exact
+                prod = np.float64(a) * xp.astype(np.float64)
+                assert np.array_equal(prod, q * xs.astype(np.float64) * 2.0 ** -69)
