@@ -62,3 +62,22 @@ def test_rejects_before_device(wq):
     assert g(P, 1, 4, 64, P, P, P, 7, 32, P, None) == wq.WQ_ERR_BITS
     assert g(P, 1, 4, 64, P, P, P, 4, 96, P, None) == wq.WQ_ERR_GROUP
     assert g(P, 1, 4, 64, P, P, P + 4, 4, 32, P, None) == wq.WQ_ERR_ALIGN
+
+
+def test_binding_checks_tensors_before_the_library(wq):
+    """The Python binding refuses host tensors, wrong dtypes and mismatched
+    shapes itself, before any pointer reaches the C ABI."""
+    import torch
+    c = torch.zeros(4, 8, dtype=torch.int32)
+    s = torch.zeros(4, 2, dtype=torch.float16)
+    x = torch.zeros(1, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        wq.wq_gemm(x, c, s, s, 4, 32, 4, 64)                      # host tensor
+    with pytest.raises(ValueError):
+        wq.wq_gemm(x.float(), c, s, s, 4, 32, 4, 64)              # not bf16
+    with pytest.raises(ValueError):
+        wq.wq_gemm(torch.zeros(64, dtype=torch.bfloat16), c, s, s, 4, 32, 4, 64)   # not 2-D
+    with pytest.raises(ValueError):
+        wq.wq_quantize_rtn(torch.zeros(4, 64, dtype=torch.float32), 4, 32)          # not fp16
+    with pytest.raises(ValueError):
+        wq.wq_quantize_rtn(torch.zeros(4, 64, dtype=torch.float16).t(), 4, 32)      # not contiguous
