@@ -106,17 +106,33 @@ wq_status wq_quantize_rtn(const void* W_f16, int64_t N, int64_t K, int bits, int
  *   y_bf16     out  bf16 [M, N] row-major; must not overlap the inputs
  *   stream          cudaStream_t
  *
- * Products and sums are fp32; y is rounded once to bf16 (RNE).  M <= 16 runs a
- * CUDA-core GEMV (codes streamed once by TMA, unpacked in registers, exact
- * x * (q - zero) products); larger M with K a multiple of 128 runs a
- * tensor-core GEMM (tcgen05 MMA, operands staged by TMA, W' dequantised to
- * bf16 in shared memory, accumulators in tensor memory), other K the GEMV 16
- * batch rows at a time.  Accuracy: every product is exact or rounded once
- * (w' to bf16 on the tensor-core path with grouped grids), sums are fp32, and
+ * Products and sums are fp32; y is rounded once to bf16 (RNE).  Which kernel
+ * runs depends on the batch M (every path streams the packed codes once and
+ * unpacks them on chip; K below means "K, and K * bits, allow TMA staging"):
+ *   M = 1        CUDA-core GEMV: codes staged by TMA, unpacked in registers,
+ *                exact x * q products (K * bits a multiple of 128);
+ *   M = 2..8     warp-level tensor-core GEMV (mma.sync, bf16 in, fp32 out):
+ *                codes unpacked in registers into the A operand, the tokens
+ *                are the MMA's columns (K and group multiples of 128);
+ *   M = 2..16    otherwise: tcgen05 GEMV with the unpacked codes in tensor
+ *                memory (K a multiple of 128; 3-bit codes need groups that
+ *                are multiples of 128), else a CUDA-core GEMV;
+ *   M > 16       tcgen05 GEMM (operands staged by TMA, W' dequantised to
+ *                bf16 in shared memory, accumulators in tensor memory) when K
+ *                is a multiple of 128, else the GEMV 16 batch rows at a time.
+ * The decode paths use tensor cores from M = 2 on because a CUDA-core dot
+ * product costs one FMA per code and token, so its cost grows with M while
+ * the bytes read do not.  Accuracy: every product is exact or rounded once
+ * (w' to bf16 on the tensor-core GEMM with grouped grids), sums are fp32, and
  * y carries one bf16 rounding (up to 2^-8 |y|); on realistic inputs each y
  * element lies within 2e-3 * sum_k |x w'| + 2^-8 |y| + 1e-3 of the exact
  * value (arithmetic error, the output rounding, an absolute floor), which is
- * the acceptance bound the tests use.  |x| must stay below 2^63.
+ * the acceptance bound the tests use.  Range of x: |x| must stay below 2^63.
+ * The decode paths form each product at a fixed power-of-two scale (2^-85 on
+ * CUDA cores, 2^-69 on the tensor cores); entries with |x| below about 2^-57
+ * give products under the fp32 normal range, which the tensor cores may flush
+ * to zero: such entries may contribute nothing, an absolute error below
+ * 2^-57 * sum_k |w'_k|, far under the 1e-3 floor.
  */
 wq_status wq_gemm(const void* x_bf16, int64_t M, int64_t N, int64_t K, const uint32_t* codes,
                   const void* scales_f16, const void* zeros_f16, int bits, int64_t group,

@@ -216,6 +216,7 @@ gemv_mma_kernel(const __grid_constant__ CUtensorMap tm_codes, const __nv_bfloat1
     // ---------------------------------------------------------------- producer
     if (lane == 0) {
       bool ok = true;
+      int ic = 0;                                   // stages issued
       for (int t = 0; t < T && ok; ++t) {
         const int s = t % D;
         if (t >= D) ok = mma_wait_bounded(empty0 + 8 * s, uint32_t(((t / D) - 1) & 1));
@@ -240,9 +241,13 @@ gemv_mma_kernel(const __grid_constant__ CUtensorMap tm_codes, const __nv_bfloat1
                   xraw0 + s * Cfg::XRAW_BYTES + m * 2048),
               "l"(x + int64_t(m) * K + k0), "r"(xbytes), "r"(full0 + 8 * s)
               : "memory");
+        ++ic;
       }
-      if (!ok) {   // copies issued but not consumed must land before the CTA exits
-        for (int t = 0; t < T; ++t) {
+      if (!ok) {
+        // Copies issued but not consumed must land before the CTA exits.  Only
+        // the last D issued stages can still be in flight (a slot is re-armed
+        // only by issuing the stage D later), each in phase t / D of its slot.
+        for (int t = ic > D ? ic - D : 0; t < ic; ++t) {
           const uint64_t t0 = now_ns();
           while (!mbar_try(full0 + 8 * (t % D), uint32_t((t / D) & 1)) && now_ns() - t0 < kWaitNs / 5) {
           }

@@ -234,3 +234,32 @@ def test_gemv_small_batch_one_hot_exact_g128(bits, M):
         ref = ((2.0 if i % 2 else -1.0) * torch.from_numpy(wq_ref[:, k])).to(torch.bfloat16)
         assert torch.equal(y[i], ref), (i, k)
     assert torch.equal(y[M - 1], torch.zeros(N, dtype=torch.bfloat16))
+
+
+def _sampled_case(seed, N, K, bits, group, M, what):
+    """Full GPU quantise + GEMV; the oracle on 128 sampled output rows."""
+    Wh = wq_inputs.weight_f16(seed, bits, N, K)
+    x = wq_inputs.activations_bf16(seed, M, M, K)
+    m = wq()
+    codes, s, z = m.wq_quantize_rtn(to_dev_f16(Wh), bits, group)
+    y = m.wq_gemm(x.cuda(), codes, s, z, bits, group, N, K).float().cpu().numpy()
+    cols = np.unique(np.concatenate([[0, N - 1], np.random.default_rng(seed).integers(0, N, 126)]))
+    oc, os_, oz = oracle_quantize(Wh[cols], bits, group)
+    y_ref, bound = oracle.gemm(wq_inputs.bf16_bits(x), oc, os_, oz, len(cols), K, bits, group)
+    assert_y_close(y[:, cols], y_ref, bound, what)
+
+
+@pytest.mark.parametrize("bits", (3, 4))
+@pytest.mark.parametrize("M", [2, 4, 8])
+def test_gemv_small_batch_split_k_cluster(bits, M):
+    """2..8 tokens, N = 4096, K = 11008, g = 128 (the 7B down projection):
+    the warp-MMA GEMV splits K over a 2-CTA cluster and adds the partial sums
+    through distributed shared memory."""
+    _sampled_case(16, 4096, 11008, bits, 128, M, f"split-K bits={bits} M={M}")
+
+
+def test_gemv_small_batch_table_windows_g128():
+    """4 tokens, N = 14240, K = 16512, g = 128: one CTA's K range spans 129
+    scale groups, more than its shared table holds, so the warp-MMA GEMV
+    reloads the table between stages."""
+    _sampled_case(17, 14240, 16512, 2, 128, 4, "warp-MMA table windows")
