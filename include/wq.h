@@ -65,7 +65,8 @@ typedef enum {
   WQ_ERR_ALIGN = 5,               /* a pointer is not 16-byte aligned */
   WQ_ERR_UNSUPPORTED_DEVICE = 6,  /* current device is not compute capability 10.0 */
   WQ_ERR_CUDA = 7,                /* a CUDA runtime call or launch failed */
-  WQ_ERR_DEVICE_TIMEOUT = 8       /* a bounded device-side wait expired (see below) */
+  WQ_ERR_DEVICE_TIMEOUT = 8,      /* a bounded device-side wait expired (see below) */
+  WQ_ERR_WORKSPACE = 9            /* workspace NULL or smaller than the call needs */
 } wq_status;
 
 /*
@@ -137,6 +138,62 @@ wq_status wq_quantize_rtn(const void* W_f16, int64_t N, int64_t K, int bits, int
 wq_status wq_gemm(const void* x_bf16, int64_t M, int64_t N, int64_t K, const uint32_t* codes,
                   const void* scales_f16, const void* zeros_f16, int bits, int64_t group,
                   void* y_bf16, void* stream);
+
+/*
+ * One linear y = x . W'^T of a grouped call: every field as for wq_gemm
+ * (x bf16 [M, K], codes/scales/zeros of W [N, K] as wq_quantize_rtn wrote
+ * them, y bf16 [M, N]).  The linears of a call share M and bits; each has its
+ * own x, shape and group.
+ */
+typedef struct {
+  const void* x_bf16;
+  const uint32_t* codes;
+  const void* scales_f16;
+  const void* zeros_f16;
+  void* y_bf16;
+  int64_t N, K, group;
+} wq_linear;
+
+/*
+ * wq_gemm_grouped -- y_l = x_l . W'_l^T for `count` independent linears in as
+ * few launches as possible (the decode step of a transformer layer stack: the
+ * same dequantise-in-the-matmul as wq_gemm, with the bandwidth argument of
+ * the BladeLLM page, "Background information > Solutions").
+ *
+ *   linears    in   host array of `count` descriptors (read during the call only)
+ *   count           >= 1
+ *   M               batch rows, common to all linears
+ *   bits            2, 3, 4 or 8, common to all linears
+ *   workspace       device buffer of at least wq_gemm_grouped_workspace_size()
+ *                   bytes, 16-byte aligned, ZERO-FILLED by the caller before
+ *                   its first use; every completed call leaves its counters
+ *                   at zero again (a call that ends in WQ_ERR_DEVICE_TIMEOUT
+ *                   may not: zero the workspace again after one).  Calls that
+ *                   share a workspace must be ordered (same stream).  May be
+ *                   NULL when the size is 0.
+ *   workspace_bytes its size
+ *   stream          cudaStream_t
+ *
+ * For M <= 16, linears whose K and group are multiples of 128 (or per-row
+ * grids with K a multiple of 128) run in one persistent kernel per 128
+ * linears: every linear is cut into 32-row tiles and 1024-code stages, the
+ * stage sequence of all linears is split evenly over the CTAs (a tile cut
+ * between two CTAs is finished through the workspace in a fixed order, so
+ * results do not depend on timing), and the codes stream through a TMA ring
+ * that never drains between tiles or linears.  A short preparation kernel
+ * first writes each x, pre-scaled for the tensor cores, into the workspace.
+ * The multiply-adds run on warp-level MMAs (mma.sync, bf16 in, fp32 out),
+ * with the same exact products and the same accuracy bound as wq_gemm.  Other
+ * linears (and every linear when M > 16) run as wq_gemm would run them.
+ * Every argument of every linear is checked before anything is launched, as
+ * for wq_gemm; outputs must not overlap any input or each other.
+ */
+wq_status wq_gemm_grouped(const wq_linear* linears, int count, int64_t M, int bits, void* workspace,
+                          size_t workspace_bytes, void* stream);
+
+/* Workspace bytes wq_gemm_grouped needs for these linears, M and bits (0 if
+ * none is needed or an argument is invalid).  Needs no device. */
+size_t wq_gemm_grouped_workspace_size(const wq_linear* linears, int count, int64_t M, int bits);
 
 /* Number of uint32 words of packed codes for an [N, K] matrix: N*K*bits/32
  * (0 if bits or K are invalid). */

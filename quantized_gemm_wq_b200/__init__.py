@@ -8,6 +8,7 @@ be loaded, importing this package fails.
 
     codes, scales, zeros = wq_quantize_rtn(W_f16, bits, group)
     y = wq_gemm(x_bf16, codes, scales, zeros, bits, group, N, K)
+    ys = wq_gemm_grouped([(x, codes, scales, zeros, N, K, group), ...], bits, workspace)
 """
 from __future__ import annotations
 
@@ -29,10 +30,19 @@ WQ_ERR_ALIGN = 5
 WQ_ERR_UNSUPPORTED_DEVICE = 6
 WQ_ERR_CUDA = 7
 WQ_ERR_DEVICE_TIMEOUT = 8
+WQ_ERR_WORKSPACE = 9
 
 # Functions the header declares (the tests check the library exports them).
-EXPORTED = ("wq_quantize_rtn", "wq_gemm", "wq_codes_words", "wq_params_count",
-            "wq_status_string", "wq_last_device_error")
+EXPORTED = ("wq_quantize_rtn", "wq_gemm", "wq_gemm_grouped", "wq_gemm_grouped_workspace_size",
+            "wq_codes_words", "wq_params_count", "wq_status_string", "wq_last_device_error")
+
+
+class Linear(ctypes.Structure):
+    """``wq_linear`` of include/wq.h: one linear of a grouped call."""
+    _fields_ = [("x_bf16", ctypes.c_void_p), ("codes", ctypes.c_void_p),
+                ("scales_f16", ctypes.c_void_p), ("zeros_f16", ctypes.c_void_p),
+                ("y_bf16", ctypes.c_void_p), ("N", ctypes.c_int64), ("K", ctypes.c_int64),
+                ("group", ctypes.c_int64)]
 
 
 def _load():
@@ -45,6 +55,11 @@ def _load():
     lib.wq_quantize_rtn.restype = ci
     lib.wq_gemm.argtypes = [vp, i64, i64, i64, vp, vp, vp, ci, i64, vp, vp]
     lib.wq_gemm.restype = ci
+    lp = ctypes.POINTER(Linear)
+    lib.wq_gemm_grouped.argtypes = [lp, ci, i64, ci, vp, ctypes.c_size_t, vp]
+    lib.wq_gemm_grouped.restype = ci
+    lib.wq_gemm_grouped_workspace_size.argtypes = [lp, ci, i64, ci]
+    lib.wq_gemm_grouped_workspace_size.restype = ctypes.c_size_t
     lib.wq_codes_words.argtypes = [i64, i64, ci]
     lib.wq_codes_words.restype = ctypes.c_size_t
     lib.wq_params_count.argtypes = [i64, i64, i64]
@@ -134,3 +149,58 @@ def wq_gemm(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, zeros: t
                      _ptr(y), _stream_ptr(stream))
     _check(st, "wq_gemm")
     return y
+
+
+def _linear_array(items, M):
+    """ctypes array of ``wq_linear`` from (x, codes, scales, zeros, N, K, group, y)
+    tuples; allocates the missing outputs."""
+    arr = (Linear * len(items))()
+    ys = []
+    for i, it in enumerate(items):
+        x, codes, scales, zeros, N, K, group = it[:7]
+        y = it[7] if len(it) > 7 and it[7] is not None else None
+        if x.dtype != torch.bfloat16 or x.dim() != 2 or not x.is_cuda or not x.is_contiguous():
+            raise ValueError("every x must be a contiguous CUDA bf16 [M, K] tensor")
+        if x.shape[0] != M or x.shape[1] != K:
+            raise ValueError("every x must be [M, K] with the call's M")
+        if y is None:
+            y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+        arr[i] = Linear(_ptr(x), _ptr(codes), _ptr(scales), _ptr(zeros), _ptr(y), N, K, group)
+        ys.append(y)
+    return arr, ys
+
+
+def grouped_workspace_size(items, bits: int) -> int:
+    """Workspace bytes ``wq_gemm_grouped`` needs for these linears."""
+    if not items:
+        return 0
+    M = items[0][0].shape[0]
+    arr, _ = _linear_array([it[:7] for it in items], M) if items[0][0].is_cuda else (None, None)
+    if arr is None:
+        raise ValueError("x must be a CUDA tensor")
+    return int(lib.wq_gemm_grouped_workspace_size(arr, len(items), M, bits))
+
+
+def grouped_workspace(items, bits: int, device=None) -> torch.Tensor:
+    """A zero-filled device workspace for ``wq_gemm_grouped`` on these linears
+    (uint8, at least 16 bytes so it always has an address)."""
+    n = grouped_workspace_size(items, bits)
+    dev = device if device is not None else items[0][0].device
+    return torch.zeros(max(16, n), dtype=torch.uint8, device=dev)
+
+
+def wq_gemm_grouped(items, bits: int, workspace=None, stream=None):
+    """``y_l = x_l . W'_l^T`` for every (x, codes, scales, zeros, N, K, group[, y])
+    of ``items`` (common M and bits) -> list of bf16 ``y_l``.  ``workspace``: a
+    zero-filled uint8 CUDA tensor from ``grouped_workspace`` (made here when
+    None; reuse one across calls on the same stream)."""
+    if not items:
+        return []
+    M = items[0][0].shape[0]
+    arr, ys = _linear_array(items, M)
+    if workspace is None:
+        workspace = grouped_workspace(items, bits)
+    st = lib.wq_gemm_grouped(arr, len(items), M, bits, _ptr(workspace),
+                             workspace.numel() * workspace.element_size(), _stream_ptr(stream))
+    _check(st, "wq_gemm_grouped")
+    return ys

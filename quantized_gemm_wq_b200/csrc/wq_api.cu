@@ -3,8 +3,10 @@
 //
 // Every check runs before any launch, so a failing call writes nothing.
 #include <mutex>
+#include <vector>
 
 #include "../../include/wq.h"
+#include "grouped.h"
 #include "wq_internal.cuh"
 
 namespace {
@@ -46,6 +48,61 @@ wq_status check_common(int64_t N, int64_t K, int bits, int64_t group) {
   return WQ_OK;
 }
 
+// One linear, arguments already checked: the kernel by batch size (see wq.h).
+cudaError_t dispatch_one(const __nv_bfloat16* x, int64_t M, int64_t N, int64_t K, const uint32_t* codes,
+                         const __half* s, const __half* z, int bits, int64_t g, __nv_bfloat16* y,
+                         cudaStream_t strm) {
+  cudaError_t e;
+  if (M > wq::kGemvMaxM && wq::gemm_tc_supported(K, bits)) {
+    e = wq::launch_gemm_tc(x, M, N, K, codes, s, z, bits, g, y, strm);
+  } else {
+    // Small batches, and K that the tensor-core GEMM cannot stage with TMA
+    // (K not a multiple of 128): 16 batch rows per launch.  One row runs the
+    // CUDA-core GEMV (its short pipeline wins at one row); 2..16 rows the
+    // tensor-core GEMVs where their shape rules allow, else the CUDA-core GEMV.
+    e = cudaSuccess;
+    for (int64_t m0 = 0; m0 < M && e == cudaSuccess; m0 += wq::kGemvMaxM) {
+      const int mc = int(M - m0 < wq::kGemvMaxM ? M - m0 : wq::kGemvMaxM);
+      if (wq::gemv_mma_supported(mc, x + m0 * K, codes, K, g))
+        e = wq::launch_gemv_mma(x + m0 * K, mc, N, K, codes, s, z, bits, g, y + m0 * N, strm);
+      else if (wq::gemv_tc_supported(mc, K, bits, g))
+        e = wq::launch_gemv_tc(x + m0 * K, mc, N, K, codes, s, z, bits, g, y + m0 * N, strm);
+      else
+        e = wq::launch_gemv(x + m0 * K, mc, N, K, codes, s, z, bits, g, y + m0 * N, strm);
+    }
+  }
+  return e;
+}
+
+// Checks of one grouped linear (same rules as wq_gemm).
+wq_status check_linear(const wq_linear& L, int64_t M, int bits) {
+  if (!L.x_bf16 || !L.codes || !L.scales_f16 || !L.zeros_f16 || !L.y_bf16) return WQ_ERR_NULL;
+  wq_status st = check_common(L.N, L.K, bits, L.group);
+  if (st != WQ_OK) return st;
+  if (M < 1 || M >= kMaxDim) return WQ_ERR_SHAPE;
+  if (!aligned16(L.x_bf16) || !aligned16(L.codes) || !aligned16(L.scales_f16) || !aligned16(L.zeros_f16) ||
+      !aligned16(L.y_bf16))
+    return WQ_ERR_ALIGN;
+  return WQ_OK;
+}
+
+wq::GroupedLinear to_grouped(const wq_linear& L) {
+  return wq::GroupedLinear{static_cast<const __nv_bfloat16*>(L.x_bf16), L.codes,
+                           static_cast<const __half*>(L.scales_f16), static_cast<const __half*>(L.zeros_f16),
+                           static_cast<__nv_bfloat16*>(L.y_bf16), L.N, L.K, wq::effective_group(L.K, L.group)};
+}
+
+// The linears of a grouped call that the persistent kernel takes.
+std::vector<wq::GroupedLinear> grouped_fast_list(const wq_linear* lins, int count, int64_t M) {
+  std::vector<wq::GroupedLinear> v;
+  if (M > wq::kGemvMaxM) return v;
+  for (int i = 0; i < count; ++i) {
+    const wq::GroupedLinear g = to_grouped(lins[i]);
+    if (wq::grouped_supported(g.K, g.group)) v.push_back(g);
+  }
+  return v;
+}
+
 }  // namespace
 
 extern "C" {
@@ -71,6 +128,7 @@ const char* wq_status_string(wq_status s) {
     case WQ_ERR_UNSUPPORTED_DEVICE: return "the current device is not compute capability 10.0 (B200)";
     case WQ_ERR_CUDA: return "a CUDA call or kernel launch failed";
     case WQ_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait expired";
+    case WQ_ERR_WORKSPACE: return "the workspace is NULL or smaller than the call needs";
   }
   return "unknown status";
 }
@@ -103,41 +161,61 @@ wq_status wq_gemm(const void* x_bf16, int64_t M, int64_t N, int64_t K, const uin
     return WQ_ERR_ALIGN;
   if ((st = check_device()) != WQ_OK) return st;
   const int64_t g = wq::effective_group(K, group);
-  const auto* x = static_cast<const __nv_bfloat16*>(x_bf16);
-  const auto* s = static_cast<const __half*>(scales_f16);
-  const auto* z = static_cast<const __half*>(zeros_f16);
-  auto* y = static_cast<__nv_bfloat16*>(y_bf16);
-  auto strm = static_cast<cudaStream_t>(stream);
-  cudaError_t e;
-  if (M > wq::kGemvMaxM && wq::gemm_tc_supported(K, bits)) {
-    e = wq::launch_gemm_tc(x, M, N, K, codes, s, z, bits, g, y, strm);
-  } else {
-    // Small batches, and K that the tensor-core GEMM cannot stage with TMA
-    // (K not a multiple of 128): 16 batch rows per launch.  One row runs the
-    // CUDA-core GEMV (its short pipeline wins at one row); 2..16 rows the
-    // tensor-core GEMV where its shape rules allow, else the CUDA-core GEMV.
-    e = cudaSuccess;
-    for (int64_t m0 = 0; m0 < M && e == cudaSuccess; m0 += wq::kGemvMaxM) {
-      const int mc = int(M - m0 < wq::kGemvMaxM ? M - m0 : wq::kGemvMaxM);
-      if (wq::gemv_mma_supported(mc, x + m0 * K, codes, K, g))
-        e = wq::launch_gemv_mma(x + m0 * K, mc, N, K, codes, s, z, bits, g, y + m0 * N, strm);
-      else if (wq::gemv_tc_supported(mc, K, bits, g))
-        e = wq::launch_gemv_tc(x + m0 * K, mc, N, K, codes, s, z, bits, g, y + m0 * N, strm);
-      else
-        e = wq::launch_gemv(x + m0 * K, mc, N, K, codes, s, z, bits, g, y + m0 * N, strm);
-    }
+  const cudaError_t e = dispatch_one(static_cast<const __nv_bfloat16*>(x_bf16), M, N, K, codes,
+                                     static_cast<const __half*>(scales_f16),
+                                     static_cast<const __half*>(zeros_f16), bits, g,
+                                     static_cast<__nv_bfloat16*>(y_bf16), static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? WQ_OK : WQ_ERR_CUDA;
+}
+
+size_t wq_gemm_grouped_workspace_size(const wq_linear* linears, int count, int64_t M, int bits) {
+  if (!linears || count < 1 || !valid_bits(bits)) return 0;
+  for (int i = 0; i < count; ++i)
+    if (check_linear(linears[i], M, bits) != WQ_OK) return 0;
+  const std::vector<wq::GroupedLinear> fast = grouped_fast_list(linears, count, M);
+  if (fast.empty()) return 0;
+  return wq::grouped_workspace_layout(fast.data(), int(fast.size()), int(M), 0, nullptr);
+}
+
+wq_status wq_gemm_grouped(const wq_linear* linears, int count, int64_t M, int bits, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+  if (!linears) return WQ_ERR_NULL;
+  if (count < 1) return WQ_ERR_SHAPE;
+  if (!valid_bits(bits)) return WQ_ERR_BITS;
+  for (int i = 0; i < count; ++i) {
+    const wq_status st = check_linear(linears[i], M, bits);
+    if (st != WQ_OK) return st;
+  }
+  const std::vector<wq::GroupedLinear> fast = grouped_fast_list(linears, count, M);
+  wq::WsLayout ws;
+  if (!fast.empty()) {
+    const size_t need = wq::grouped_workspace_layout(fast.data(), int(fast.size()), int(M), 0, nullptr);
+    if (!workspace || workspace_bytes < need) return WQ_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return WQ_ERR_ALIGN;
+    wq::grouped_workspace_layout(fast.data(), int(fast.size()), int(M), reinterpret_cast<uintptr_t>(workspace),
+                                 &ws);
+  }
+  wq_status st = check_device();
+  if (st != WQ_OK) return st;
+  const auto strm = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaSuccess;
+  if (!fast.empty()) e = wq::launch_gemv_grouped(fast.data(), int(fast.size()), int(M), bits, ws, strm);
+  for (int i = 0; i < count && e == cudaSuccess; ++i) {
+    const wq::GroupedLinear g = to_grouped(linears[i]);
+    if (M <= wq::kGemvMaxM && wq::grouped_supported(g.K, g.group)) continue;
+    e = dispatch_one(g.x, M, g.N, g.K, g.codes, g.scales, g.zeros, bits, g.group, g.y, strm);
   }
   return e == cudaSuccess ? WQ_OK : WQ_ERR_CUDA;
 }
 
 wq_status wq_last_device_error(void) {
-  cudaError_t e1 = cudaSuccess, e2 = cudaSuccess, e3 = cudaSuccess, e4 = cudaSuccess;
-  const bool hit1 = wq::gemm_tc_read_and_clear_timeout(&e1);
-  const bool hit2 = wq::gemv_m1_tma_read_and_clear_timeout(&e2);
-  const bool hit3 = wq::gemv_tc_read_and_clear_timeout(&e3);
-  const bool hit4 = wq::gemv_mma_read_and_clear_timeout(&e4);
-  if (e1 != cudaSuccess || e2 != cudaSuccess || e3 != cudaSuccess || e4 != cudaSuccess) return WQ_ERR_CUDA;
-  return (hit1 || hit2 || hit3 || hit4) ? WQ_ERR_DEVICE_TIMEOUT : WQ_OK;
+  cudaError_t e[5] = {cudaSuccess, cudaSuccess, cudaSuccess, cudaSuccess, cudaSuccess};
+  const bool hit = wq::gemm_tc_read_and_clear_timeout(&e[0]) | wq::gemv_m1_tma_read_and_clear_timeout(&e[1]) |
+                   wq::gemv_tc_read_and_clear_timeout(&e[2]) | wq::gemv_mma_read_and_clear_timeout(&e[3]) |
+                   wq::gemv_grouped_read_and_clear_timeout(&e[4]);
+  for (cudaError_t x : e)
+    if (x != cudaSuccess) return WQ_ERR_CUDA;
+  return hit ? WQ_ERR_DEVICE_TIMEOUT : WQ_OK;
 }
 
 }  // extern "C"

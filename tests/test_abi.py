@@ -40,7 +40,7 @@ def test_layout_helpers(wq):
 
 
 def test_status_strings(wq):
-    for s in range(9):
+    for s in range(10):
         assert len(wq.wq_status_string(s)) >= 2
     assert "unknown" in wq.wq_status_string(99)
 
@@ -81,3 +81,35 @@ def test_binding_checks_tensors_before_the_library(wq):
         wq.wq_quantize_rtn(torch.zeros(4, 64, dtype=torch.float32), 4, 32)          # not fp16
     with pytest.raises(ValueError):
         wq.wq_quantize_rtn(torch.zeros(4, 64, dtype=torch.float16).t(), 4, 32)      # not contiguous
+
+
+def test_grouped_rejects_before_device(wq):
+    """wq_gemm_grouped checks every linear and the workspace before touching
+    the device; its workspace size needs no device."""
+    L = wq.lib
+    P = 1 << 20
+
+    def lin(N=64, K=1024, group=128, x=P, z=P):
+        return wq.Linear(x, P, P, z, P, N, K, group)
+
+    arr = (wq.Linear * 2)(lin(), lin(N=96, K=2048, group=0))
+    n1 = L.wq_gemm_grouped_workspace_size(arr, 2, 1, 4)
+    n16 = L.wq_gemm_grouped_workspace_size(arr, 2, 16, 4)
+    assert 0 < n1 < n16
+    assert L.wq_gemm_grouped_workspace_size(arr, 2, 17, 4) == 0          # M > 16: no workspace
+    assert L.wq_gemm_grouped_workspace_size(arr, 2, 1, 5) == 0           # bad bits
+    small = (wq.Linear * 1)(lin(K=96, group=32))                         # not the persistent kernel's shape
+    assert L.wq_gemm_grouped_workspace_size(small, 1, 1, 4) == 0
+    assert L.wq_gemm_grouped(arr, 2, 1, 4, None, 0, None) == wq.WQ_ERR_WORKSPACE
+    assert L.wq_gemm_grouped(arr, 2, 1, 4, P, n1 - 1, None) == wq.WQ_ERR_WORKSPACE
+    assert L.wq_gemm_grouped(arr, 2, 1, 4, P + 8, n1, None) == wq.WQ_ERR_ALIGN
+    assert L.wq_gemm_grouped(None, 2, 1, 4, P, n1, None) == wq.WQ_ERR_NULL
+    assert L.wq_gemm_grouped(arr, 0, 1, 4, P, n1, None) == wq.WQ_ERR_SHAPE
+    assert L.wq_gemm_grouped(arr, 2, 0, 4, P, n1, None) == wq.WQ_ERR_SHAPE
+    assert L.wq_gemm_grouped(arr, 2, 1, 7, P, n1, None) == wq.WQ_ERR_BITS
+    bad = (wq.Linear * 2)(lin(), lin(group=96))
+    assert L.wq_gemm_grouped(bad, 2, 1, 4, P, n1, None) == wq.WQ_ERR_GROUP
+    bad = (wq.Linear * 2)(lin(), lin(x=P + 2))
+    assert L.wq_gemm_grouped(bad, 2, 1, 4, P, n1, None) == wq.WQ_ERR_ALIGN
+    bad = (wq.Linear * 2)(lin(), lin(K=100))
+    assert L.wq_gemm_grouped(bad, 2, 1, 4, P, n1, None) == wq.WQ_ERR_SHAPE
