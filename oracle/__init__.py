@@ -12,6 +12,9 @@ Parity status of each function (what pins it, see ``tests/test_oracle.py``):
   midpoints by exact arithmetic).
 * ``quantize_rtn``: pinned (closed-form designed grids, brute-force nearest grid
   point in exact rational arithmetic, exact rational scale/zero, invariants).
+* ``quantize_rtn_sym``: pinned (designed symmetric grids, brute-force nearest
+  grid point in exact rational arithmetic, exact rational scale, odd symmetry,
+  invariants).
 * ``pack`` / ``unpack``: pinned (hand-derived words in ``tests/golden``,
   round trips).
 * ``dequant`` / ``gemm``: pinned (exact rational sums on tiny inputs, one-hot
@@ -41,6 +44,8 @@ def _lib():
             getattr(lib, name).restype = None
         lib.orc_quantize_rtn.argtypes = [_p, _i64, _i64, ctypes.c_int, _i64, _p, _p, _p, ctypes.c_int]
         lib.orc_quantize_rtn.restype = ctypes.c_int
+        lib.orc_quantize_rtn_sym.argtypes = [_p, _i64, _i64, ctypes.c_int, _i64, _p, _p, ctypes.c_int]
+        lib.orc_quantize_rtn_sym.restype = ctypes.c_int
         lib.orc_pack.argtypes = [_p, _i64, _i64, ctypes.c_int, _p]
         lib.orc_pack.restype = ctypes.c_int
         lib.orc_unpack.argtypes = [_p, _i64, _i64, ctypes.c_int, _p]
@@ -117,6 +122,27 @@ def quantize_rtn(W_bits, bits: int, group: int, nthreads: int = 0):
     if rc != 0:
         raise OracleError(f"invalid arguments N={N} K={K} bits={bits} group={group}")
     return q, s, z
+
+
+def quantize_rtn_sym(W_bits, bits: int, group: int, nthreads: int = 0):
+    """Round-to-nearest quantisation on the symmetric grid (zero fixed at
+    2^(bits-1), not stored).  Returns ``(q, scales)``."""
+    W = _c(W_bits, np.uint16)
+    N, K = W.shape
+    G = groups_per_row(K, group) if K % 32 == 0 and (group in (0, K) or (group > 0 and K % group == 0)) else 1
+    q = np.empty((N, K), np.uint8)
+    s = np.empty((N, G), np.uint16)
+    rc = _lib().orc_quantize_rtn_sym(_ptr(W), N, K, bits, group, _ptr(q), _ptr(s), nthreads)
+    if rc != 0:
+        raise OracleError(f"invalid arguments N={N} K={K} bits={bits} group={group}")
+    return q, s
+
+
+def sym_zeros(scales, bits: int):
+    """The zeros a symmetric grid implies: fp16 bit patterns of 2^(bits-1), the
+    shape of ``scales`` (what ``dequant`` and ``gemm`` take)."""
+    s = np.asarray(scales)
+    return np.full(s.shape, f64_to_f16(np.array([float(1 << (bits - 1))]))[0], np.uint16)
 
 
 def pack(q, bits: int):

@@ -35,6 +35,13 @@
 //   R5 zero is not clamped; it is a non-negative integer stored exactly in fp16,
 //      with a clear sign bit;
 //   R6 group 0 or group K means one (scale, zero) per row;
+//   S1 the symmetric grid ("Platform For AI: BladeLLM model quantization",
+//      "Quantization modes > weight_only_quant": signed symmetric quantisation
+//      by default): a = max |w| over the group, scale = fp16 RNE of
+//      a / (2^(b-1) - 1) (1 if that is 0), the zero fixed at 2^(b-1) and not
+//      stored; the codes are the same RTN codes on that grid, so the signed
+//      value q - 2^(b-1) of +-a is +-(2^(b-1) - 1), and the extra code 0 is
+//      only reached by rounding or a scale rounded down;
 //   R7 packing is LSB-first along K: for b in {2,4,8} code k sits in word
 //      k / (32/b) at bit b*(k mod 32/b); for b = 3 the 32 codes of unit
 //      u = k/32 fill the 96-bit little-endian value of words 3u..3u+2, code
@@ -229,6 +236,35 @@ int orc_quantize_rtn(const uint16_t* W, int64_t N, int64_t K, int bits, int64_t 
       }
       scales[n * G + j] = to_f16(s);
       zeros[n * G + j] = to_f16(z);
+      for (int64_t k = j * g; k < (j + 1) * g; ++k) {
+        double c = std::nearbyint(f16(wr[k]) / s) + z;
+        c = std::min(std::max(c, 0.0), qmax);
+        q[n * K + k] = uint8_t(c);
+      }
+    }
+  });
+  return 0;
+}
+
+// ------------------------------------------------ quantise, symmetric grid (S1)
+// Same layout as orc_quantize_rtn; no zeros output (every zero is 2^(b-1)).
+int orc_quantize_rtn_sym(const uint16_t* W, int64_t N, int64_t K, int bits, int64_t group,
+                         uint8_t* q, uint16_t* scales, int nthreads) {
+  if (!W || !q || !scales || N < 1 || K < 1 || K % 32 != 0 || !valid_bits(bits)) return -1;
+  const int64_t g = effective_group(K, group);
+  if (g < 0) return -1;
+  const int64_t G = K / g;
+  const double qmax = double((1 << bits) - 1);
+  const double z = double(1 << (bits - 1));
+  const double top = z - 1.0;                 // signed code of +a
+  parallel_rows(N, nthreads, [&](int64_t n) {
+    const uint16_t* wr = W + n * K;
+    for (int64_t j = 0; j < G; ++j) {
+      double a = 0.0;
+      for (int64_t k = j * g; k < (j + 1) * g; ++k) a = std::max(a, std::fabs(f16(wr[k])));
+      double s = f16(to_f16(a / top));
+      if (s == 0.0) s = 1.0;                  // all-zero group or underflow (as R4)
+      scales[n * G + j] = to_f16(s);
       for (int64_t k = j * g; k < (j + 1) * g; ++k) {
         double c = std::nearbyint(f16(wr[k]) / s) + z;
         c = std::min(std::max(c, 0.0), qmax);
