@@ -92,6 +92,24 @@ wq_status wq_quantize_rtn(const void* W_f16, int64_t N, int64_t K, int bits, int
                           uint32_t* codes, void* scales_f16, void* zeros_f16, void* stream);
 
 /*
+ * wq_quantize_rtn_sym -- round-to-nearest quantisation on the symmetric grid
+ * ("Platform For AI: BladeLLM model quantization", "Quantization modes >
+ * weight_only_quant": signed symmetric quantisation is the default; groups as
+ * in "block_wise_quant").  Per row or group:
+ *
+ *   a = max |w|,  scale = fp16_rne(a / (2^(b-1) - 1))  (1.0 if that rounds to 0)
+ *   zero = 2^(b-1) (fixed, not stored)
+ *   q = clamp(rint(w / scale) + 2^(b-1), 0, 2^b - 1),   w' = scale * (q - 2^(b-1))
+ *
+ * so +-a map to the signed codes +-(2^(b-1) - 1).  Arguments as for
+ * wq_quantize_rtn, without zeros_f16.  Pass zeros_f16 = NULL to wq_gemm and
+ * wq_gemm_grouped for codes written by this call.  Bit-exact like
+ * wq_quantize_rtn (the scale divisor 2^(b-1) - 1 is this library's reading).
+ */
+wq_status wq_quantize_rtn_sym(const void* W_f16, int64_t N, int64_t K, int bits, int64_t group,
+                              uint32_t* codes, void* scales_f16, void* stream);
+
+/*
  * wq_gemm -- y = x . W'^T with W' dequantised on the fly from the codes.
  * (Dequantise-in-the-matmul: onnxruntime issue 14997, weights kept in 4 bit and
  * converted to float when used; BladeLLM page, "Background information >
@@ -102,7 +120,8 @@ wq_status wq_quantize_rtn(const void* W_f16, int64_t N, int64_t K, int bits, int
  *   M, N, K         batch rows, output features, input features
  *   codes      in   packed codes as written by wq_quantize_rtn
  *   scales_f16 in   fp16 [N, G]
- *   zeros_f16  in   fp16 [N, G]
+ *   zeros_f16  in   fp16 [N, G], or NULL for the symmetric grid of
+ *                   wq_quantize_rtn_sym (every zero 2^(bits-1))
  *   bits, group     as given to wq_quantize_rtn
  *   y_bf16     out  bf16 [M, N] row-major; must not overlap the inputs
  *   stream          cudaStream_t
@@ -142,8 +161,8 @@ wq_status wq_gemm(const void* x_bf16, int64_t M, int64_t N, int64_t K, const uin
 /*
  * One linear y = x . W'^T of a grouped call: every field as for wq_gemm
  * (x bf16 [M, K], codes/scales/zeros of W [N, K] as wq_quantize_rtn wrote
- * them, y bf16 [M, N]).  The linears of a call share M and bits; each has its
- * own x, shape and group.
+ * them, zeros NULL for a symmetric grid, y bf16 [M, N]).  The linears of a
+ * call share M and bits; each has its own x, shape, group and grid.
  */
 typedef struct {
   const void* x_bf16;

@@ -33,7 +33,7 @@ WQ_ERR_DEVICE_TIMEOUT = 8
 WQ_ERR_WORKSPACE = 9
 
 # Functions the header declares (the tests check the library exports them).
-EXPORTED = ("wq_quantize_rtn", "wq_gemm", "wq_gemm_grouped", "wq_gemm_grouped_workspace_size",
+EXPORTED = ("wq_quantize_rtn", "wq_quantize_rtn_sym", "wq_gemm", "wq_gemm_grouped", "wq_gemm_grouped_workspace_size",
             "wq_codes_words", "wq_params_count", "wq_status_string", "wq_last_device_error")
 
 
@@ -53,6 +53,8 @@ def _load():
     i64, vp, ci = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int
     lib.wq_quantize_rtn.argtypes = [vp, i64, i64, ci, i64, vp, vp, vp, vp]
     lib.wq_quantize_rtn.restype = ci
+    lib.wq_quantize_rtn_sym.argtypes = [vp, i64, i64, ci, i64, vp, vp, vp]
+    lib.wq_quantize_rtn_sym.restype = ci
     lib.wq_gemm.argtypes = [vp, i64, i64, i64, vp, vp, vp, ci, i64, vp, vp]
     lib.wq_gemm.restype = ci
     lp = ctypes.POINTER(Linear)
@@ -135,9 +137,26 @@ def wq_quantize_rtn(W: torch.Tensor, bits: int, group: int, codes=None, scales=N
     return codes, scales, zeros
 
 
-def wq_gemm(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, zeros: torch.Tensor,
+def wq_quantize_rtn_sym(W: torch.Tensor, bits: int, group: int, codes=None, scales=None, stream=None):
+    """Quantise fp16 ``W`` [N, K] (CUDA) on the symmetric grid (zero 2^(bits-1),
+    not stored) -> (codes, scales, None); pass the None as ``zeros``."""
+    if W.dtype != torch.float16 or W.dim() != 2 or not W.is_cuda or not W.is_contiguous():
+        raise ValueError("W must be a contiguous CUDA fp16 [N, K] tensor")
+    N, K = W.shape
+    G = groups_per_row(K, group) if group in (0, K) or (group > 0 and K % group == 0) else 1
+    if codes is None:
+        codes = torch.empty((N, max(1, K * bits // 32)), dtype=torch.int32, device=W.device)
+    if scales is None:
+        scales = torch.empty((N, G), dtype=torch.float16, device=W.device)
+    st = lib.wq_quantize_rtn_sym(_ptr(W), N, K, bits, group, _ptr(codes), _ptr(scales), _stream_ptr(stream))
+    _check(st, "wq_quantize_rtn_sym")
+    return codes, scales, None
+
+
+def wq_gemm(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, zeros,
             bits: int, group: int, N: int, K: int, y=None, stream=None) -> torch.Tensor:
-    """``y = x . W'^T`` for bf16 ``x`` [M, K] (CUDA) -> bf16 ``y`` [M, N]."""
+    """``y = x . W'^T`` for bf16 ``x`` [M, K] (CUDA) -> bf16 ``y`` [M, N];
+    ``zeros`` None for codes of the symmetric grid."""
     if x.dtype != torch.bfloat16 or x.dim() != 2 or not x.is_cuda or not x.is_contiguous():
         raise ValueError("x must be a contiguous CUDA bf16 [M, K] tensor")
     M = x.shape[0]

@@ -405,7 +405,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
     for (int i = 0; i < 2; ++i) {
       const int64_t n = n0 + r0 + 16 * i;
       srow[i] = n < N ? reinterpret_cast<const unsigned short*>(scales) + n * G : nullptr;
-      zrow[i] = n < N ? reinterpret_cast<const unsigned short*>(zeros) + n * G : nullptr;
+      zrow[i] = n < N && zeros ? reinterpret_cast<const unsigned short*>(zeros) + n * G : nullptr;
     }
     auto load_raw = [&](int kt, uint16_t (&s2)[2], uint16_t (&z2)[2]) {
       const int k = kt * BK + 32 * cu;
@@ -416,7 +416,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         z2[i] = 0;
         if (kt < kt1 && srow[i] != nullptr && k < K) {
           s2[i] = rowwise ? uint16_t(0x3C00) : __ldg(srow[i] + grp);   // 0x3C00: fp16 1.0
-          z2[i] = __ldg(zrow[i] + grp);
+          // no zeros array: the symmetric grid's zero 2^(b-1) as fp16 bits
+          z2[i] = zrow[i] ? __ldg(zrow[i] + grp) : uint16_t((BITS - 1 + 15) << 10);
         }
       }
     };

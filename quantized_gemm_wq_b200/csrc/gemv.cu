@@ -210,7 +210,7 @@ __device__ __forceinline__ void load_step(Step<BITS, R>& st, const uint32_t* __r
     if (u < KU && n < N) {
       load_unit<BITS>(codes + n * KW + u * BITS, st.w[r]);
       st.s[r] = __half2float(scales[n * G + grp]);
-      st.z[r] = __half2float(zeros[n * G + grp]);
+      st.z[r] = zeros ? __half2float(zeros[n * G + grp]) : float(1 << (BITS - 1));
     } else {
 #pragma unroll
       for (int i = 0; i < BITS; ++i) st.w[r][i] = 0u;
@@ -304,7 +304,7 @@ gemvm_kernel(const __nv_bfloat16* __restrict__ x, int M, int64_t N, int64_t K,
       if (n < N) {
         load_unit<BITS>(codes + n * KW + u * BITS, w);
         sc[r] = __half2float(scales[n * G + grp]);
-        zz[r] = __half2float(zeros[n * G + grp]);
+        zz[r] = zeros ? __half2float(zeros[n * G + grp]) : float(1 << (BITS - 1));
       } else {
 #pragma unroll
         for (int i = 0; i < BITS; ++i) w[i] = 0u;

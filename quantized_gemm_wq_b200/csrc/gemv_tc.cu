@@ -254,7 +254,12 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __nv_bfloat16* __
     {
       const __half* src = h ? zeros : scales;
       uint32_t* dst = sstage + (h * kRows + row) * kSPitch;
-      if (n < N) {
+      if (n < N && src == nullptr) {
+        // no zeros array (symmetric grid): every zero is 2^(b-1)
+        constexpr uint32_t zh = uint32_t(BITS - 1 + 15) << 10;
+        int wi = 0;
+        for (int64_t a = e0 - off; a <= n * G + gB; a += 2, ++wi) dst[wi] = zh | (zh << 16);
+      } else if (n < N) {
         const int64_t total = N * G;
         int wi = 0;
         for (int64_t a = e0 - off; a <= n * G + gB; a += 2, ++wi) {

@@ -196,7 +196,7 @@ gemv_m1_tma_kernel(const __grid_constant__ CUtensorMap tm_codes, const __nv_bflo
     const int trow = threadIdx.x >> 3, tj = threadIdx.x & 7;
     const bool trow_in = row0 + trow < N;
     const __half* srow = scales + (trow_in ? row0 + trow : 0) * G;
-    const __half* zrow = zeros + (trow_in ? row0 + trow : 0) * G;
+    const __half* zrow = zeros ? zeros + (trow_in ? row0 + trow : 0) * G : nullptr;
     auto load_table = [&](int64_t wg0) {
       float sv[16], zv[16];
 #pragma unroll
@@ -204,7 +204,7 @@ gemv_m1_tma_kernel(const __grid_constant__ CUtensorMap tm_codes, const __nv_bflo
         const int j = tj + 8 * i;
         const bool in = trow_in && j < gcap && wg0 + j < G;
         sv[i] = in ? __half2float(srow[wg0 + j]) : 0.0f;
-        zv[i] = in ? __half2float(zrow[wg0 + j]) : 0.0f;
+        zv[i] = in ? (zrow ? __half2float(zrow[wg0 + j]) : float(1 << (BITS - 1))) : 0.0f;
       }
       asm volatile("bar.sync 1, %0;" ::"n"(32 * NW) : "memory");   // old table no longer read
 #pragma unroll

@@ -92,17 +92,27 @@ struct Grid {
   __half sh;
 };
 
+// Asymmetric grid (sym false): scale from the range [lo, hi], zero rint(-lo /
+// scale).  Symmetric grid (sym true; "Platform For AI: BladeLLM model
+// quantization", "Quantization modes > weight_only_quant": signed symmetric by
+// default): a = max(-lo, hi) = max |w|, scale = fp16(a / (2^(b-1) - 1)), zero
+// fixed at 2^(b-1) and not stored.  One fp64 division then one RNE to fp16
+// equals exact rounding for the divisors 1, 3, 7, 127 as for 3, 7, 15, 255.
 template <int BITS>
-__device__ __forceinline__ Grid make_grid(float lo, float hi) {
+__device__ __forceinline__ Grid make_grid(float lo, float hi, bool sym) {
   constexpr double qmax = double((1 << BITS) - 1);
-  const double d = (double(hi) - double(lo)) / qmax;  // exact difference, one rounding
+  constexpr double top = double((1 << (BITS - 1)) - 1);
+  const double d = sym ? double(fmaxf(0.0f - lo, hi)) / top
+                       : (double(hi) - double(lo)) / qmax;   // exact difference, one rounding
   Grid gr;
   gr.sh = __double2half(d);                           // one RNE to fp16
   gr.s = __half2float(gr.sh);
   if (gr.s == 0.0f) {                                  // degenerate range
     gr.s = 1.0f;
     gr.sh = __float2half_rn(1.0f);
-    gr.z = 0.0f;
+    gr.z = sym ? float(1 << (BITS - 1)) : 0.0f;
+  } else if (sym) {
+    gr.z = float(1 << (BITS - 1));
   } else {
     gr.z = rintf(__fdiv_rn(0.0f - lo, gr.s));          // 0 - lo is never -0
   }
@@ -159,10 +169,10 @@ quantize_small_kernel(const __half* __restrict__ W, int64_t nseg, int64_t K, int
     hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, off, TPS));
   }
   if (!active) return;
-  const Grid gr = make_grid<BITS>(lo, hi);
+  const Grid gr = make_grid<BITS>(lo, hi, zeros == nullptr);
   if (sub == 0) {
     scales[seg] = gr.sh;
-    zeros[seg] = __float2half_rn(gr.z);
+    if (zeros) zeros[seg] = __float2half_rn(gr.z);
   }
   for (int blk = sub; blk < nblk; blk += TPS) {
     Block32 b;
@@ -213,10 +223,10 @@ quantize_large_kernel(const __half* __restrict__ W, int64_t K, int64_t g,
     lo = fminf(lo, s_lo[w]);
     hi = fmaxf(hi, s_hi[w]);
   }
-  const Grid gr = make_grid<BITS>(lo, hi);
+  const Grid gr = make_grid<BITS>(lo, hi, zeros == nullptr);
   if (threadIdx.x == 0) {
     scales[seg] = gr.sh;
-    zeros[seg] = __float2half_rn(gr.z);
+    if (zeros) zeros[seg] = __float2half_rn(gr.z);
   }
   for (int blk = threadIdx.x; blk < nblk; blk += kThreads) {
     Block32 b;

@@ -76,12 +76,12 @@ cudaError_t dispatch_one(const __nv_bfloat16* x, int64_t M, int64_t N, int64_t K
 
 // Checks of one grouped linear (same rules as wq_gemm).
 wq_status check_linear(const wq_linear& L, int64_t M, int bits) {
-  if (!L.x_bf16 || !L.codes || !L.scales_f16 || !L.zeros_f16 || !L.y_bf16) return WQ_ERR_NULL;
+  if (!L.x_bf16 || !L.codes || !L.scales_f16 || !L.y_bf16) return WQ_ERR_NULL;   // zeros NULL: symmetric
   wq_status st = check_common(L.N, L.K, bits, L.group);
   if (st != WQ_OK) return st;
   if (M < 1 || M >= kMaxDim) return WQ_ERR_SHAPE;
-  if (!aligned16(L.x_bf16) || !aligned16(L.codes) || !aligned16(L.scales_f16) || !aligned16(L.zeros_f16) ||
-      !aligned16(L.y_bf16))
+  if (!aligned16(L.x_bf16) || !aligned16(L.codes) || !aligned16(L.scales_f16) ||
+      (L.zeros_f16 && !aligned16(L.zeros_f16)) || !aligned16(L.y_bf16))
     return WQ_ERR_ALIGN;
   return WQ_OK;
 }
@@ -149,15 +149,30 @@ wq_status wq_quantize_rtn(const void* W_f16, int64_t N, int64_t K, int bits, int
   return e == cudaSuccess ? WQ_OK : WQ_ERR_CUDA;
 }
 
+wq_status wq_quantize_rtn_sym(const void* W_f16, int64_t N, int64_t K, int bits, int64_t group,
+                              uint32_t* codes, void* scales_f16, void* stream) {
+  if (!W_f16 || !codes || !scales_f16) return WQ_ERR_NULL;
+  wq_status st = check_common(N, K, bits, group);
+  if (st != WQ_OK) return st;
+  if (!aligned16(W_f16) || !aligned16(codes) || !aligned16(scales_f16)) return WQ_ERR_ALIGN;
+  if ((st = check_device()) != WQ_OK) return st;
+  // a null zeros array selects the symmetric grid in the quantiser
+  cudaError_t e = wq::launch_quantize(static_cast<const __half*>(W_f16), N, K, bits,
+                                      wq::effective_group(K, group), codes,
+                                      static_cast<__half*>(scales_f16), nullptr,
+                                      static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? WQ_OK : WQ_ERR_CUDA;
+}
+
 wq_status wq_gemm(const void* x_bf16, int64_t M, int64_t N, int64_t K, const uint32_t* codes,
                   const void* scales_f16, const void* zeros_f16, int bits, int64_t group,
                   void* y_bf16, void* stream) {
-  if (!x_bf16 || !codes || !scales_f16 || !zeros_f16 || !y_bf16) return WQ_ERR_NULL;
+  if (!x_bf16 || !codes || !scales_f16 || !y_bf16) return WQ_ERR_NULL;   // zeros NULL: symmetric grid
   wq_status st = check_common(N, K, bits, group);
   if (st != WQ_OK) return st;
   if (M < 1 || M >= kMaxDim) return WQ_ERR_SHAPE;
   if (!aligned16(x_bf16) || !aligned16(codes) || !aligned16(scales_f16) ||
-      !aligned16(zeros_f16) || !aligned16(y_bf16))
+      (zeros_f16 && !aligned16(zeros_f16)) || !aligned16(y_bf16))
     return WQ_ERR_ALIGN;
   if ((st = check_device()) != WQ_OK) return st;
   const int64_t g = wq::effective_group(K, group);

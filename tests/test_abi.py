@@ -113,3 +113,23 @@ def test_grouped_rejects_before_device(wq):
     assert L.wq_gemm_grouped(bad, 2, 1, 4, P, n1, None) == wq.WQ_ERR_ALIGN
     bad = (wq.Linear * 2)(lin(), lin(K=100))
     assert L.wq_gemm_grouped(bad, 2, 1, 4, P, n1, None) == wq.WQ_ERR_SHAPE
+
+
+def test_symmetric_entry_points_reject_before_device(wq):
+    """wq_quantize_rtn_sym checks its arguments like wq_quantize_rtn; a NULL
+    zeros pointer is the symmetric grid for wq_gemm, not an error."""
+    L = wq.lib
+    P = 1 << 20
+    q = L.wq_quantize_rtn_sym
+    assert q(None, 4, 64, 4, 32, P, P, None) == wq.WQ_ERR_NULL
+    assert q(P, 4, 64, 4, 32, P, None, None) == wq.WQ_ERR_NULL
+    assert q(P, 4, 64, 6, 32, P, P, None) == wq.WQ_ERR_BITS
+    assert q(P, 4, 63, 4, 0, P, P, None) == wq.WQ_ERR_SHAPE
+    assert q(P, 4, 64, 4, 48, P, P, None) == wq.WQ_ERR_GROUP
+    assert q(P, 4, 64, 4, 32, P + 4, P, None) == wq.WQ_ERR_ALIGN
+    g = L.wq_gemm
+    st = g(P, 1, 4, 64, P, P, None, 4, 32, P, None)
+    assert st not in (wq.WQ_ERR_NULL, wq.WQ_ERR_ALIGN, wq.WQ_ERR_SHAPE, wq.WQ_ERR_GROUP, wq.WQ_ERR_BITS)
+    assert g(P, 1, 4, 64, P, None, None, 4, 32, P, None) == wq.WQ_ERR_NULL     # scales are required
+    arr = (wq.Linear * 1)(wq.Linear(P, P, P, None, P, 64, 1024, 128))
+    assert L.wq_gemm_grouped_workspace_size(arr, 1, 1, 4) > 0

@@ -54,8 +54,10 @@ def test_two_gloo_ranks_max_and_aggregate():
 def test_step_bytes_headline():
     sys.path.insert(0, ROOT)
     import bench
-    # 3-bit codes + fp16 scale/zero per 128 inputs + x + y of the four projections
+    # 32 layers of q, k, v, o 4096->4096, gate, up 4096->11008, down 11008->4096:
+    # 4-bit codes + fp16 scale/zero per 128 inputs + x + y
     exp = 0
-    for N, K in [(12288, 4096), (4096, 4096), (22016, 4096), (4096, 11008)]:
-        exp += N * K * 3 // 8 + N * (K // 128) * 4 + K * 2 + N * 2
-    assert bench.step_bytes(bench.HEADLINE, 1) == exp
+    for N, K in [(4096, 4096)] * 4 + [(11008, 4096)] * 2 + [(4096, 11008)]:
+        exp += N * K * 4 // 8 + N * (K // 128) * 4 + K * 2 + N * 2
+    assert bench.step_bytes(bench.HEADLINE, 1) == 32 * exp
+    assert abs(32 * exp / 1e9 - 3.44) < 0.01
