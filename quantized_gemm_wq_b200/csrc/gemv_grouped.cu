@@ -22,8 +22,10 @@
 //           workspace, written by xprep_kernel): for token m and code slot k,
 //           x 2^(64 - b), b the code's bit offset in its 16-bit half;
 //   sum x   per 128-code quad and token (bulk copy from the workspace);
-//   (s, z)  of the stage's scale groups for the 32 rows, loaded by the 32
-//           lanes of the producer warp one stage ahead and stored as floats.
+//   (s, z)  the raw fp16 scales and zeros of the stage's groups for the 32
+//           rows: each lane of the producer warp copies its row's window with
+//           4-byte cp.async copies that arrive on the same barrier when they
+//           land, so the producer never waits for them.
 // Warp 8 is the producer; warps 0..7 consume, warp w quad w of every stage,
 // exactly as in the 2..8-token GEMV (gemv_mma.cu): lane (g, t) unpacks unit
 // 4w + t of rows g, g + 8, g + 16, g + 24 with one AND per two codes into the
@@ -56,7 +58,11 @@ using namespace stg;
 constexpr uint64_t kWaitNs = 1000000000ull;   // 1 s: far beyond any healthy wait
 constexpr int kNW = 8;                        // consumer warps
 constexpr int kThreads = 32 * (kNW + 1);
-constexpr int kSzRow = 9;                     // float2 per row of an (s, z) slot: 8 groups + pad
+// Words per row of an (s, z) slot: up to 9 halves of scales (8 groups and an
+// odd start) in 5 words, then 5 words of zeros.  10 words apart, the rows
+// g = 0..7 a consumer lane reads fall in distinct banks.
+constexpr int kSzW = 5;
+constexpr int kSzRow = 2 * kSzW;
 
 __device__ __noinline__ bool wait_bounded(uint32_t bar, uint32_t parity) {
   if (mbar_try(bar, parity)) return true;
@@ -196,7 +202,7 @@ struct GCfg {
   static constexpr int SB = BITS * 4096;                  // codes: 32 rows x 32 units
   static constexpr int XB = MT * 2048;                    // x': 8 quads x MT tokens x 256 B
   static constexpr int SXB = 8 * Tok<MT>::SXW * 4;        // sums per quad and token
-  static constexpr int SZB = 32 * kSzRow * 8;             // (s, z) of 32 rows x up to 8 groups
+  static constexpr int SZB = 32 * kSzRow * 4;             // raw (s, z) of 32 rows x up to 8 groups
   static constexpr int RB = MT <= 8 ? 2 : 1;              // tile reduction buffers
   static constexpr int REDB = RB * kNW * MT * 32 * 4;
   static constexpr int OFF_XP = D * SB;
@@ -253,7 +259,9 @@ __global__ void __launch_bounds__(kThreads, MINB) gemv_grouped_kernel(const __gr
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < D; ++s) {
-      asm volatile("mbarrier.init.shared::cta.b64 [%0], 2;" ::"r"(full0 + 8 * s));
+      // full: the producer's expect-tx arrive + one arrive per producer lane
+      // (its scale/zero copies)
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 33;" ::"r"(full0 + 8 * s));
       asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(empty0 + 8 * s), "r"(kNW));
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -265,27 +273,51 @@ __global__ void __launch_bounds__(kThreads, MINB) gemv_grouped_kernel(const __gr
   if (warp == kNW) {
     // ------------------------------------------------------------ producer
     Pos q = locate(p, sb);
-    float sv[8], zv[8];
-    int gs = 0;
-    // (s, z) of the stage at q for row 32 r + lane, groups [gfirst, gfirst + gs)
-    auto load_sz = [&](const Pos& at) {
+    // This lane's row of the stage's scales and zeros into the slot: the
+    // halves [e0, e0 + gs) of each array, copied as the aligned 4-byte words
+    // that hold them (word w at slot word w, zeros 5 words later).  A window
+    // whose last word would pass the end of the arrays is read with plain
+    // loads instead.  Every lane arrives on the stage's full barrier once.
+    auto copy_sz = [&](const Pos& at, uint32_t full, uint32_t sz_slot) {
       const GLin& L = p.lin[at.l];
       const int64_t n = at.r * 32 + lane;
+      if (n >= L.N) {
+        asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(full) : "memory");
+        return;
+      }
       const int KU = L.K / 32;
       const uint32_t u0 = uint32_t(at.t) * 32, ul = uint32_t(min(at.t * 32 + 32, KU) - 1);
-      const int gfirst = int(L.upg.div(u0));
-      gs = int(L.upg.div(ul)) - gfirst + 1;
-      const bool in = n < L.N;
-      const __half* sr = L.scales + (in ? n : 0) * L.G + gfirst;
-      const __half* zr = L.zeros ? L.zeros + (in ? n : 0) * L.G + gfirst : nullptr;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const bool v = in && j < gs;
-        sv[j] = v ? __half2float(sr[j]) : 0.0f;
-        zv[j] = v ? (zr ? __half2float(zr[j]) : float(1 << (BITS - 1))) : 0.0f;
+      const int64_t gfirst = L.upg.div(u0);
+      const int gs = int(L.upg.div(ul) - gfirst) + 1;
+      const int64_t e0 = n * L.G + gfirst, a0 = e0 & ~int64_t(1);
+      const int nw = int((e0 + gs - a0 + 1) >> 1);
+      const uint32_t sw = sz_slot + uint32_t(lane * kSzRow * 4);
+      if (a0 + 2 * nw <= int64_t(L.N) * L.G) {
+        const uint32_t* sg = reinterpret_cast<const uint32_t*>(L.scales + a0);
+        const uint32_t* zg = L.zeros ? reinterpret_cast<const uint32_t*>(L.zeros + a0) : nullptr;
+        for (int w = 0; w < nw; ++w) {
+          asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(sw + 4 * w), "l"(sg + w) : "memory");
+          if (zg)
+            asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(sw + 4 * (kSzW + w)), "l"(zg + w)
+                         : "memory");
+        }
+        asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(full) : "memory");
+      } else {
+        const unsigned short* sh = reinterpret_cast<const unsigned short*>(L.scales);
+        const unsigned short* zh = reinterpret_cast<const unsigned short*>(L.zeros);
+        const int64_t end = int64_t(L.N) * L.G;
+        for (int w = 0; w < nw; ++w) {
+          const int64_t a = a0 + 2 * w;
+          const uint32_t lo = a < end ? sh[a] : 0u, hi = a + 1 < end ? sh[a + 1] : 0u;
+          asm volatile("st.shared.u32 [%0], %1;" ::"r"(sw + 4 * w), "r"(lo | (hi << 16)) : "memory");
+          if (zh) {
+            const uint32_t zl = a < end ? zh[a] : 0u, zu = a + 1 < end ? zh[a + 1] : 0u;
+            asm volatile("st.shared.u32 [%0], %1;" ::"r"(sw + 4 * (kSzW + w)), "r"(zl | (zu << 16)) : "memory");
+          }
+        }
+        asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(full) : "memory");
       }
     };
-    load_sz(q);
     bool ok = true;
     int ic = 0;
     for (int i = 0; i < T; ++i) {
@@ -323,17 +355,10 @@ __global__ void __launch_bounds__(kThreads, MINB) gemv_grouped_kernel(const __gr
             "l"(L.sx + int64_t(q.t) * 8 * SXW), "r"(sxb), "r"(full0 + 8 * s)
             : "memory");
       }
-      float2* szr = reinterpret_cast<float2*>(smem + C::OFF_SZ + s * C::SZB) + lane * kSzRow;
-#pragma unroll
-      for (int j = 0; j < 8; ++j)
-        if (j < gs) szr[j] = make_float2(sv[j], zv[j]);
-      __syncwarp();
-      if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(full0 + 8 * s) : "memory");
+      const uint32_t sz_slot_s = ring + C::OFF_SZ + s * C::SZB;
+      copy_sz(q, full0 + 8 * s, sz_slot_s);
       ++ic;
-      if (i + 1 < T) {
-        advance(p, q);
-        load_sz(q);
-      }
+      if (i + 1 < T) advance(p, q);
     }
     if (!ok && lane == 0) {
       // Copies issued but not consumed must land before the CTA exits: only
@@ -432,11 +457,20 @@ __global__ void __launch_bounds__(kThreads, MINB) gemv_grouped_kernel(const __gr
       const int gq = int(L.upg.div(uq));
       const bool next_in = !seg_end && kq + 1024 < L.K;
       if (!next_in || int(L.upg.div(uq + 32)) != gq) {
-        const int rel = gq - int(L.upg.div(uint32_t(q.t) * 32));
-        const float2* sz = reinterpret_cast<const float2*>(smem + C::OFF_SZ + s * C::SZB) + rel;
+        // (s, z) of rows g + 8 r: half (e0 & 1) + rel of the row's window,
+        // e0 = n G + gfirst its first needed half (see the producer)
+        const int64_t gfirst = L.upg.div(uint32_t(q.t) * 32);
+        const int rel = int(gq - gfirst);
+        const __half* szs = reinterpret_cast<const __half*>(smem + C::OFF_SZ + s * C::SZB);
         float2 zs[4];
 #pragma unroll
-        for (int r = 0; r < 4; ++r) zs[r] = sz[(g + 8 * r) * kSzRow];
+        for (int r = 0; r < 4; ++r) {
+          const int row = g + 8 * r;
+          const int h = int(((q.r * 32 + row) * L.G + gfirst) & 1) + rel;
+          const __half* rs = szs + row * (2 * kSzRow);
+          zs[r].x = __half2float(rs[h]);
+          zs[r].y = L.zeros ? __half2float(rs[2 * kSzW + h]) : float(1 << (BITS - 1));
+        }
         // rows g, g + 8 from cA (cA2), rows g + 16, g + 24 from cB (cB2)
         const float dv[4][4] = {{cA[0], cA[1], cA2[0], cA2[1]},
                                 {cA[2], cA[3], cA2[2], cA2[3]},
