@@ -1,5 +1,10 @@
 """Build ``libwq.so`` (the C-ABI library) in-tree with nvcc for sm_100a.
 
+A second build, ``libwq_shortwait.so``, compiles the same sources with a
+pipeline-wait limit of 0 (``WQ_PIPE_WAIT_NS``): every bounded wait that is not
+already complete expires at once.  Only the tests load it, to check that an
+expired wait is reported as WQ_ERR_DEVICE_TIMEOUT and leaves the GPU usable.
+
 Each ``csrc/*.cu`` translation unit is compiled for ``sm_100a`` only, the CUDA
 runtime is linked statically and the CUDA driver API is reached at run time
 through ``cudaGetDriverEntryPoint``, so the library loads on a host without a
@@ -17,6 +22,11 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libwq.so")
+VARIANTS = {"": [], "shortwait": ["-DWQ_PIPE_WAIT_NS=0ull"]}
+
+
+def lib_path(variant: str = "") -> str:
+    return os.path.join(HERE, f"libwq_{variant}.so" if variant else "libwq.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
@@ -32,21 +42,25 @@ def _deps():
         [os.path.join(HERE, "..", "include", "wq.h"), __file__]
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB):
+def _stale(lib: str) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return any(os.path.getmtime(p) > t for p in _deps())
 
 
-def build(force: bool = False, verbose: bool = False, extra=()) -> str:
-    if not force and not _stale():
-        return LIB
-    os.makedirs(BUILD, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, extra=(), variant: str = "") -> str:
+    """Build one library (``variant`` "" for libwq.so); returns its path."""
+    lib = lib_path(variant)
+    if not force and not _stale(lib):
+        return lib
+    bdir = os.path.join(BUILD, variant) if variant else BUILD
+    os.makedirs(bdir, exist_ok=True)
+    vflags = VARIANTS[variant]
 
     def compile_one(src):
-        obj = os.path.join(BUILD, os.path.basename(src) + ".o")
-        cmd = [NVCC, *ARCH, *FLAGS, *extra, "-c", src, "-o", obj]
+        obj = os.path.join(bdir, os.path.basename(src) + ".o")
+        cmd = [NVCC, *ARCH, *FLAGS, *vflags, *extra, "-c", src, "-o", obj]
         if verbose:
             cmd.insert(1, "-Xptxas=-v")
         r = subprocess.run(cmd, capture_output=True, text=True)
@@ -60,15 +74,21 @@ def build(force: bool = False, verbose: bool = False, extra=()) -> str:
         for _, err in results:
             sys.stderr.write(err)
     objs = [o for o, _ in results]
-    tmp = LIB + f".tmp{os.getpid()}"
+    tmp = lib + f".tmp{os.getpid()}"
     cmd = [NVCC, *ARCH, "-shared", "-cudart", "static", "-Xcompiler", "-fPIC",
            "-Xlinker", "--no-undefined", *objs, "-o", tmp, "-ldl", "-lpthread", "-lrt"]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
+
+
+def build_all(force: bool = False) -> None:
+    for v in VARIANTS:
+        build(force=force, variant=v)
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))
+    for v in VARIANTS:
+        print(build(force="--force" in sys.argv, verbose="-v" in sys.argv, variant=v))

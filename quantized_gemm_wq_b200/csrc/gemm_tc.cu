@@ -32,6 +32,7 @@
 
 #include <atomic>
 
+#include "bounded_wait.cuh"
 #include "wq_internal.cuh"
 
 namespace wq {
@@ -55,8 +56,6 @@ constexpr int kThreads = 64 + 32 * kDqWarps;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kABytes = BM * BK * 2;
 constexpr uint32_t kBBytes = BN * BK * 2;
-constexpr uint64_t kWaitNs = 1000000000ull;      // 1 s: far beyond any healthy wait
-constexpr uint64_t kDrainNs = 200000000ull;      // 0.2 s for the exit path
 
 template <int BITS>
 struct TcCfg {
@@ -89,49 +88,13 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t* b, uint32_t bytes) {
                "r"(bytes)
                : "memory");
 }
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* b, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(b)), "r"(parity)
-      : "memory");
-  return ok != 0;
+// Waits: bounded_wait.cuh (pipeline waits give up after its limit, raising
+// the CTA abort word and g_timeout_flag; exit-path drains ignore the abort).
+__device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, volatile uint32_t* abort) {
+  return bw::pipe_wait(smem_u32(b), parity, &g_timeout_flag, abort);
 }
-__device__ __forceinline__ uint64_t global_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-
-// Bounded wait.  Returns false if the CTA has aborted or the wait expired (the
-// latter raises the CTA abort word and the device flag).
-__device__ __noinline__ bool mbar_wait(uint64_t* b, uint32_t parity, volatile uint32_t* abort) {
-  if (mbar_try_wait(b, parity)) return true;
-  const uint64_t t0 = global_ns();
-  for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait(b, parity)) return true;
-    if ((i & 63u) == 0) {
-      if (*abort) return false;
-      if (global_ns() - t0 > kWaitNs) {
-        *abort = 1u;
-        atomicExch(&g_timeout_flag, 1u);
-        return false;
-      }
-    }
-  }
-}
-// Exit-path wait for copies still in flight: ignores the abort word.
-__device__ __noinline__ void mbar_drain(uint64_t* b, uint32_t parity) {
-  const uint64_t t0 = global_ns();
-  while (!mbar_try_wait(b, parity)) {
-    if (global_ns() - t0 > kDrainNs) {
-      atomicExch(&g_timeout_flag, 1u);
-      return;
-    }
-  }
+__device__ __forceinline__ void mbar_drain(uint64_t* b, uint32_t parity) {
+  bw::drain_wait(smem_u32(b), parity, &g_timeout_flag);
 }
 
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar,

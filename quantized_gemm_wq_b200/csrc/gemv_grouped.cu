@@ -55,7 +55,6 @@ namespace {
 
 using namespace stg;
 
-constexpr uint64_t kWaitNs = 1000000000ull;   // 1 s: far beyond any healthy wait
 constexpr int kNW = 8;                        // consumer warps
 constexpr int kThreads = 32 * (kNW + 1);
 // Words per row of an (s, z) slot: up to 9 halves of scales (8 groups and an
@@ -64,16 +63,8 @@ constexpr int kThreads = 32 * (kNW + 1);
 constexpr int kSzW = 5;
 constexpr int kSzRow = 2 * kSzW;
 
-__device__ __noinline__ bool wait_bounded(uint32_t bar, uint32_t parity) {
-  if (mbar_try(bar, parity)) return true;
-  const uint64_t t0 = now_ns();
-  while (!mbar_try(bar, parity)) {
-    if (now_ns() - t0 > kWaitNs) {
-      atomicExch(&g_gemv_grouped_timeout, 1u);
-      return false;
-    }
-  }
-  return true;
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity) {
+  return bw::pipe_wait(bar, parity, &g_gemv_grouped_timeout, nullptr);
 }
 
 template <int BITS>
@@ -363,11 +354,8 @@ __global__ void __launch_bounds__(kThreads, MINB) gemv_grouped_kernel(const __gr
     if (!ok && lane == 0) {
       // Copies issued but not consumed must land before the CTA exits: only
       // the last D issued stages can still be in flight, each in phase t / D.
-      for (int t = ic > D ? ic - D : 0; t < ic; ++t) {
-        const uint64_t t0 = now_ns();
-        while (!mbar_try(full0 + 8 * (t % D), uint32_t((t / D) & 1)) && now_ns() - t0 < kWaitNs / 5) {
-        }
-      }
+      for (int t = ic > D ? ic - D : 0; t < ic; ++t)
+        bw::drain_wait(full0 + 8 * (t % D), uint32_t((t / D) & 1), &g_gemv_grouped_timeout);
     }
     return;
   }

@@ -52,20 +52,10 @@ using namespace stg;
 #ifndef WQ_GEMV_MMA_MIN_STAGES
 #define WQ_GEMV_MMA_MIN_STAGES 4
 #endif
-constexpr uint64_t kWaitNs = 1000000000ull;
-
 __device__ unsigned int g_gemv_mma_timeout;
 
-__device__ __noinline__ bool mma_wait_bounded(uint32_t bar, uint32_t parity) {
-  if (mbar_try(bar, parity)) return true;
-  const uint64_t t0 = now_ns();
-  while (!mbar_try(bar, parity)) {
-    if (now_ns() - t0 > kWaitNs) {
-      atomicExch(&g_gemv_mma_timeout, 1u);
-      return false;
-    }
-  }
-  return true;
+__device__ __forceinline__ bool mma_wait_bounded(uint32_t bar, uint32_t parity) {
+  return bw::pipe_wait(bar, parity, &g_gemv_mma_timeout, nullptr);
 }
 
 template <int BITS, int MT>
@@ -247,11 +237,8 @@ gemv_mma_kernel(const __grid_constant__ CUtensorMap tm_codes, const __nv_bfloat1
         // Copies issued but not consumed must land before the CTA exits.  Only
         // the last D issued stages can still be in flight (a slot is re-armed
         // only by issuing the stage D later), each in phase t / D of its slot.
-        for (int t = ic > D ? ic - D : 0; t < ic; ++t) {
-          const uint64_t t0 = now_ns();
-          while (!mbar_try(full0 + 8 * (t % D), uint32_t((t / D) & 1)) && now_ns() - t0 < kWaitNs / 5) {
-          }
-        }
+        for (int t = ic > D ? ic - D : 0; t < ic; ++t)
+          bw::drain_wait(full0 + 8 * (t % D), uint32_t((t / D) & 1), &g_gemv_mma_timeout);
       }
     }
   } else {

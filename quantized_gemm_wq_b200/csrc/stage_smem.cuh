@@ -4,28 +4,16 @@
 #pragma once
 #include <cstdint>
 
+#include "bounded_wait.cuh"
+
 namespace wq {
 namespace stg {
 
 __device__ __forceinline__ uint32_t saddr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
-__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-__device__ __forceinline__ uint64_t now_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) { return bw::try_parity(bar, parity); }
+__device__ __forceinline__ uint64_t now_ns() { return bw::now_ns(); }
 // Shared-memory byte offset of word wi (0 .. 32*BITS-1) of row r in a stage:
 // the stage holds BITS boxes of 32 words per row; inside a box, rows are 128
 // bytes apart and the 16-byte chunk index is XOR-ed with r % 8 (128B swizzle).

@@ -5,11 +5,11 @@
 #include <cuda.h>
 #include <cstdint>
 
+#include "bounded_wait.cuh"
+
 namespace wq {
 namespace ptx {
 
-constexpr uint64_t kWaitNs = 1000000000ull;   // 1 s: far beyond any healthy wait
-constexpr uint64_t kDrainNs = 200000000ull;   // 0.2 s for exit paths
 
 static __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -26,49 +26,19 @@ static __device__ __forceinline__ void mbar_expect_tx(uint64_t* b, uint32_t byte
                : "memory");
 }
 static __device__ __forceinline__ bool mbar_try_wait(uint64_t* b, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(b)), "r"(parity)
-      : "memory");
-  return ok != 0;
+  return bw::try_parity(smem_u32(b), parity);
 }
-static __device__ __forceinline__ uint64_t global_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
+static __device__ __forceinline__ uint64_t global_ns() { return bw::now_ns(); }
 
-// Bounded wait.  Returns false if the CTA has aborted or the wait expired; the
-// latter raises the CTA abort word and the kernel's device flag.
-static __device__ __noinline__ bool mbar_wait(uint64_t* b, uint32_t parity,
-                                              volatile uint32_t* abort, unsigned int* flag) {
-  if (mbar_try_wait(b, parity)) return true;
-  const uint64_t t0 = global_ns();
-  for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait(b, parity)) return true;
-    if ((i & 63u) == 0) {
-      if (*abort) return false;
-      if (global_ns() - t0 > kWaitNs) {
-        *abort = 1u;
-        atomicExch(flag, 1u);
-        return false;
-      }
-    }
-  }
+// Bounded pipeline wait (bounded_wait.cuh): false if the CTA has aborted or
+// the wait expired; the latter raises the CTA abort word and the kernel's flag.
+static __device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, volatile uint32_t* abort,
+                                                 unsigned int* flag) {
+  return bw::pipe_wait(smem_u32(b), parity, flag, abort);
 }
 // Exit-path wait for asynchronous work still in flight: ignores the abort word.
-static __device__ __noinline__ void mbar_drain(uint64_t* b, uint32_t parity, unsigned int* flag) {
-  const uint64_t t0 = global_ns();
-  while (!mbar_try_wait(b, parity)) {
-    if (global_ns() - t0 > kDrainNs) {
-      atomicExch(flag, 1u);
-      return;
-    }
-  }
+static __device__ __forceinline__ void mbar_drain(uint64_t* b, uint32_t parity, unsigned int* flag) {
+  bw::drain_wait(smem_u32(b), parity, flag);
 }
 
 static __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar,
