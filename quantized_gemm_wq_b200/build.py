@@ -1,8 +1,9 @@
 """Build ``libwq.so`` (the C-ABI library) in-tree with nvcc for sm_100a.
 
 A second build, ``libwq_shortwait.so``, compiles the same sources with a
-pipeline-wait limit of 0 (``WQ_PIPE_WAIT_NS``): every bounded wait that is not
-already complete expires at once.  Only the tests load it, to check that an
+pipeline-wait limit of 0 (``WQ_PIPE_WAIT_NS``) and the test hook
+``wq_test_expire_wait`` (``WQ_TEST_HOOKS``): a kernel whose bounded wait is on
+a barrier nothing arrives on.  Only the tests load it, to check that an
 expired wait is reported as WQ_ERR_DEVICE_TIMEOUT and leaves the GPU usable.
 
 Each ``csrc/*.cu`` translation unit is compiled for ``sm_100a`` only, the CUDA
@@ -22,7 +23,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libwq.so")
-VARIANTS = {"": [], "shortwait": ["-DWQ_PIPE_WAIT_NS=0ull"]}
+VARIANTS = {"": [], "shortwait": ["-DWQ_PIPE_WAIT_NS=0ull", "-DWQ_TEST_HOOKS"]}
 
 
 def lib_path(variant: str = "") -> str:

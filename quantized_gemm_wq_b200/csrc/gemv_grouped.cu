@@ -99,19 +99,64 @@ __device__ __forceinline__ void mma_bf16(float (&c)[4], uint32_t a0, uint32_t a1
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// The 8 MMAs of one 16-row tile over a quad: rows g (words wa) and g + 8
-// (words wb) of this lane's unit against one 8-token B operand (xb); with
-// TWO, the same A fragments also meet a second 8-token operand (xb2).
-template <int BITS, int J, bool TWO>
+// Accumulators of a lane for one quad: [tile][chain][4], tile 0 the rows of
+// the lane's first A fragment pair (words w[0], w[1]), tile 1 the next
+// (w[2], w[3]); chain J % 2, so consecutive MMAs of a tile do not wait for
+// each other.  `h` selects the second 8-token half (16 tokens only).
+struct QuadAcc {
+  float c[2][2][4];
+};
+
+// MMA J..7 of 16-row tile T over a quad (A rows from the words wa, wb)
+// against one 8-token B operand (xb); with TWO the same A fragments also meet
+// the second 8-token operand (xb2).
+template <int BITS, int T, int J, bool TWO>
 struct QuadMma {
-  __device__ __forceinline__ static void run(float (&c)[4], float (&c2)[4], const uint32_t (&wa)[BITS],
+  __device__ __forceinline__ static void run(QuadAcc& a, QuadAcc& a2, const uint32_t (&wa)[BITS],
                                              const uint32_t (&wb)[BITS], const uint32_t (&xb)[16],
                                              const uint32_t (&xb2)[16]) {
     const uint32_t a0 = unit_pair<BITS, 2 * J>(wa), a1 = unit_pair<BITS, 2 * J>(wb);
-    const uint32_t a2 = unit_pair<BITS, 2 * J + 1>(wa), a3 = unit_pair<BITS, 2 * J + 1>(wb);
-    mma_bf16(c, a0, a1, a2, a3, xb[2 * J], xb[2 * J + 1]);
-    if constexpr (TWO) mma_bf16(c2, a0, a1, a2, a3, xb2[2 * J], xb2[2 * J + 1]);
-    if constexpr (J + 1 < 8) QuadMma<BITS, J + 1, TWO>::run(c, c2, wa, wb, xb, xb2);
+    const uint32_t a2r = unit_pair<BITS, 2 * J + 1>(wa), a3 = unit_pair<BITS, 2 * J + 1>(wb);
+    mma_bf16(a.c[T][J & 1], a0, a1, a2r, a3, xb[2 * J], xb[2 * J + 1]);
+    if constexpr (TWO) mma_bf16(a2.c[T][J & 1], a0, a1, a2r, a3, xb2[2 * J], xb2[2 * J + 1]);
+    if constexpr (J + 1 < 8) QuadMma<BITS, T, J + 1, TWO>::run(a, a2, wa, wb, xb, xb2);
+  }
+};
+
+// Weight row (within an 8-row group) fed to MMA row g: an order in which the
+// 8 lanes of each quarter-warp load 8 distinct 16-byte bank groups from the
+// 128-byte-swizzled code boxes (2-bit and 4-bit units; 3-bit and 8-bit
+// units are conflict-free in the plain order).
+template <int BITS>
+__host__ __device__ constexpr int mma_row(int g) {
+  if constexpr (BITS == 4) return (g >> 1) | ((g & 1) << 2);
+  else if constexpr (BITS == 2) return ((g & 1) << 2) | (g & 2) | ((g >> 2) & 1);
+  else return g;
+}
+
+// The fields of the linear a CTA is working on, in registers.
+struct LinRegs {
+  const __half* scales;
+  const __half* zeros;
+  __nv_bfloat16* y;
+  const uint32_t* xp;
+  const float* sx;
+  int64_t stage0;
+  int N, K, G, TS, tiles;
+  FastDiv upg;
+  __device__ __forceinline__ void load(const GLin& L) {
+    scales = L.scales;
+    zeros = L.zeros;
+    y = L.y;
+    xp = L.xp;
+    sx = L.sx;
+    stage0 = L.stage0;
+    N = L.N;
+    K = L.K;
+    G = L.G;
+    TS = L.TS;
+    tiles = L.tiles;
+    upg = L.upg;
   }
 };
 
@@ -219,15 +264,6 @@ __device__ __forceinline__ Pos locate(const GParams& p, int64_t s) {
   const int TS = p.lin[l].TS;
   return Pos{l, int(off % TS), off / TS};
 }
-__device__ __forceinline__ void advance(const GParams& p, Pos& q) {
-  if (++q.t == p.lin[q.l].TS) {
-    q.t = 0;
-    if (++q.r == p.lin[q.l].tiles) {
-      q.r = 0;
-      ++q.l;
-    }
-  }
-}
 // First stage of CTA c's range.
 __device__ __forceinline__ int64_t range_start(const GParams& p, int64_t c) { return p.total * c / p.P; }
 
@@ -264,13 +300,14 @@ __global__ void __launch_bounds__(kThreads, MINB) gemv_grouped_kernel(const __gr
   if (warp == kNW) {
     // ------------------------------------------------------------ producer
     Pos q = locate(p, sb);
+    LinRegs L;
+    L.load(p.lin[q.l]);
     // This lane's row of the stage's scales and zeros into the slot: the
     // halves [e0, e0 + gs) of each array, copied as the aligned 4-byte words
     // that hold them (word w at slot word w, zeros 5 words later).  A window
     // whose last word would pass the end of the arrays is read with plain
     // loads instead.  Every lane arrives on the stage's full barrier once.
     auto copy_sz = [&](const Pos& at, uint32_t full, uint32_t sz_slot) {
-      const GLin& L = p.lin[at.l];
       const int64_t n = at.r * 32 + lane;
       if (n >= L.N) {
         asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(full) : "memory");
@@ -320,7 +357,6 @@ __global__ void __launch_bounds__(kThreads, MINB) gemv_grouped_kernel(const __gr
         if (!ok) break;
       }
       __syncwarp();
-      const GLin& L = p.lin[q.l];
       if (lane == 0) {
         const int rem = L.K - q.t * 1024;
         const int nq = rem >= 1024 ? 8 : rem / 128;
@@ -349,7 +385,13 @@ __global__ void __launch_bounds__(kThreads, MINB) gemv_grouped_kernel(const __gr
       const uint32_t sz_slot_s = ring + C::OFF_SZ + s * C::SZB;
       copy_sz(q, full0 + 8 * s, sz_slot_s);
       ++ic;
-      if (i + 1 < T) advance(p, q);
+      if (++q.t == L.TS) {
+        q.t = 0;
+        if (++q.r == L.tiles) {
+          q.r = 0;
+          if (++q.l < p.nlin && i + 1 < T) L.load(p.lin[q.l]);
+        }
+      }
     }
     if (!ok && lane == 0) {
       // Copies issued but not consumed must land before the CTA exits: only
@@ -363,9 +405,14 @@ __global__ void __launch_bounds__(kThreads, MINB) gemv_grouped_kernel(const __gr
   // -------------------------------------------------------------- consumers
   const int g = lane >> 2, tq = lane & 3;
   const int tid = int(threadIdx.x);
+  // this lane's rows of the 32-row tile: the MMA rows g, g + 8 of tile 0 and
+  // of tile 1 (rows 16..31) map to weight rows rw[0..3]
+  int rw[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) rw[i] = mma_row<BITS>(g) + 8 * i;
   uint32_t uoff[4][unit_pieces<BITS>()];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) unit_offsets<BITS>(g + 8 * i, 4 * warp + tq, uoff[i]);
+  for (int i = 0; i < 4; ++i) unit_offsets<BITS>(rw[i], 4 * warp + tq, uoff[i]);
   // B fragment chunk offsets in the quad's x' area: token g (and g + 8);
   // token columns past the batch tile read the zero block.
   uint32_t boffA[4], boffB[4];
@@ -380,24 +427,33 @@ __global__ void __launch_bounds__(kThreads, MINB) gemv_grouped_kernel(const __gr
   auto tok_of = [&](int c) { return 2 * tq + (c & 1) + 8 * (c >> 1); };
 
   Pos q = locate(p, sb);
+  LinRegs L;
+  L.load(p.lin[q.l]);
   float acc[4][NC];
-  float cA[4], cB[4], cA2[4], cB2[4];   // tiles rows g.. / g+16..; second 8-token half
+  QuadAcc qa, qa2;
   float sxg[NC];
+  auto zero_quad = [&]() {
 #pragma unroll
-  for (int r = 0; r < 4; ++r) {
-    cA[r] = cB[r] = cA2[r] = cB2[r] = 0.0f;
+    for (int t = 0; t < 2; ++t)
+#pragma unroll
+      for (int j = 0; j < 2; ++j)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) qa.c[t][j][e] = qa2.c[t][j][e] = 0.0f;
+#pragma unroll
+    for (int c = 0; c < NC; ++c) sxg[c] = 0.0f;
+  };
+  zero_quad();
+#pragma unroll
+  for (int r = 0; r < 4; ++r)
 #pragma unroll
     for (int c = 0; c < NC; ++c) acc[r][c] = 0.0f;
-  }
-#pragma unroll
-  for (int c = 0; c < NC; ++c) sxg[c] = 0.0f;
   bool ok = true;
   int tcount = 0;
   int64_t seg_start = sb;      // first stage of this CTA in the current tile
+  const __half hz = __float2half_rn(float(1 << (BITS - 1)));
 
   for (int i = 0; i < T; ++i) {
     const int s = i % D;
-    const GLin& L = p.lin[q.l];
     {
       const uint32_t par = uint32_t((i / D) & 1);
       if (ok) ok = __all_sync(0xffffffffu, mbar_try(full0 + 8 * s, par) || wait_bounded(full0 + 8 * s, par));
@@ -432,47 +488,47 @@ __global__ void __launch_bounds__(kThreads, MINB) gemv_grouped_kernel(const __gr
         uint32_t wa[BITS], wb[BITS];
         load_unit_at<BITS>(stage, uoff[0], wa);
         load_unit_at<BITS>(stage, uoff[1], wb);
-        QuadMma<BITS, 0, MT == 16>::run(cA, cA2, wa, wb, xa, xb2);
+        QuadMma<BITS, 0, 0, MT == 16>::run(qa, qa2, wa, wb, xa, xb2);
       }
       {
         uint32_t wa[BITS], wb[BITS];
         load_unit_at<BITS>(stage, uoff[2], wa);
         load_unit_at<BITS>(stage, uoff[3], wb);
-        QuadMma<BITS, 0, MT == 16>::run(cB, cB2, wa, wb, xa, xb2);
+        QuadMma<BITS, 1, 0, MT == 16>::run(qa, qa2, wa, wb, xa, xb2);
       }
       // fold into y when the next quad of this warp is in another group, or absent
       const uint32_t uq = uint32_t(kq / 32);
       const int gq = int(L.upg.div(uq));
       const bool next_in = !seg_end && kq + 1024 < L.K;
       if (!next_in || int(L.upg.div(uq + 32)) != gq) {
-        // (s, z) of rows g + 8 r: half (e0 & 1) + rel of the row's window,
-        // e0 = n G + gfirst its first needed half (see the producer)
-        const int64_t gfirst = L.upg.div(uint32_t(q.t) * 32);
-        const int rel = int(gq - gfirst);
+        // (s, z) of row rw[r]: half (e0 & 1) + rel of the row's window, e0 =
+        // n G + gfirst its first needed half (see the producer)
+        const int gfirst = int(L.upg.div(uint32_t(q.t) * 32));
+        const int rel = gq - gfirst;
         const __half* szs = reinterpret_cast<const __half*>(smem + C::OFF_SZ + s * C::SZB);
+        // e0 = n G + gfirst has the parity of gfirst, plus that of n when G is odd
+        const int gpar = L.G & 1;
         float2 zs[4];
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
-          const int row = g + 8 * r;
-          const int h = int(((q.r * 32 + row) * L.G + gfirst) & 1) + rel;
-          const __half* rs = szs + row * (2 * kSzRow);
+          const int h = ((gpar * (int(q.r) * 32 + rw[r]) + gfirst) & 1) + rel;
+          const __half* rs = szs + rw[r] * (2 * kSzRow);
           zs[r].x = __half2float(rs[h]);
-          zs[r].y = L.zeros ? __half2float(rs[2 * kSzW + h]) : float(1 << (BITS - 1));
+          zs[r].y = __half2float(L.zeros ? rs[2 * kSzW + h] : hz);
         }
-        // rows g, g + 8 from cA (cA2), rows g + 16, g + 24 from cB (cB2)
-        const float dv[4][4] = {{cA[0], cA[1], cA2[0], cA2[1]},
-                                {cA[2], cA[3], cA2[2], cA2[3]},
-                                {cB[0], cB[1], cB2[0], cB2[1]},
-                                {cB[2], cB[3], cB2[2], cB2[3]}};
+        // rows rw[0], rw[1] from tile 0 (MMA rows g, g + 8), rw[2], rw[3] from tile 1
 #pragma unroll
-        for (int r = 0; r < 4; ++r)
+        for (int r = 0; r < 4; ++r) {
+          const int t = r >> 1, e = 2 * (r & 1);
 #pragma unroll
-          for (int c = 0; c < NC; ++c)
-            acc[r][c] = fmaf(zs[r].x, fmaf(dv[r][c], 0x1p69f, -zs[r].y * sxg[c]), acc[r][c]);
-#pragma unroll
-        for (int r = 0; r < 4; ++r) cA[r] = cB[r] = cA2[r] = cB2[r] = 0.0f;
-#pragma unroll
-        for (int c = 0; c < NC; ++c) sxg[c] = 0.0f;
+          for (int c = 0; c < NC; ++c) {
+            const QuadAcc& src = (c >> 1) ? qa2 : qa;
+            const int ce = e + (c & 1);
+            const float d = src.c[t][0][ce] + src.c[t][1][ce];
+            acc[r][c] = fmaf(zs[r].x, fmaf(d, 0x1p69f, -zs[r].y * sxg[c]), acc[r][c]);
+          }
+        }
+        zero_quad();
       }
     }
     __syncwarp();
@@ -485,7 +541,7 @@ __global__ void __launch_bounds__(kThreads, MINB) gemv_grouped_kernel(const __gr
       for (int c = 0; c < NC; ++c)
         if (tok_of(c) < MT) {
 #pragma unroll
-          for (int r = 0; r < 4; ++r) rb[(warp * MT + tok_of(c)) * 32 + g + 8 * r] = acc[r][c];
+          for (int r = 0; r < 4; ++r) rb[(warp * MT + tok_of(c)) * 32 + rw[r]] = acc[r][c];
         }
       asm volatile("bar.sync 1, %0;" ::"n"(32 * kNW) : "memory");
       const int64_t tb = L.stage0 + q.r * L.TS, te = tb + L.TS;
@@ -497,7 +553,7 @@ __global__ void __launch_bounds__(kThreads, MINB) gemv_grouped_kernel(const __gr
         const int m = idx >> 5, row = idx & 31;
         float v = 0.0f;
 #pragma unroll
-        for (int w = 0; w < kNW; ++w) v += rb[(w * MT + m) * 32 + row];
+        for (int wv = 0; wv < kNW; ++wv) v += rb[(wv * MT + m) * 32 + row];
         if (whole) {
           if (m < p.M && row0 + row < L.N) L.y[int64_t(m) * L.N + row0 + row] = __float2bfloat16_rn(v);
         } else {
@@ -535,7 +591,14 @@ __global__ void __launch_bounds__(kThreads, MINB) gemv_grouped_kernel(const __gr
         for (int c = 0; c < NC; ++c) acc[r][c] = 0.0f;
       seg_start = sb + i + 1;
     }
-    advance(p, q);
+    // next stage; a new linear's fields are read once
+    if (++q.t == L.TS) {
+      q.t = 0;
+      if (++q.r == L.tiles) {
+        q.r = 0;
+        if (++q.l < p.nlin && i + 1 < T) L.load(p.lin[q.l]);
+      }
+    }
   }
 }
 
@@ -696,6 +759,24 @@ cudaError_t launch_gemv_grouped(const GroupedLinear* lins, int count, int M, int
   }
 }
 
+#ifdef WQ_TEST_HOOKS
+// Test builds only: one thread waits, with the library's bounded pipeline
+// wait, on a fresh mbarrier that nothing ever arrives on.  The wait runs out
+// after the build's pipeline limit and raises this file's device flag, which
+// wq_last_device_error reports; nothing faults and nothing is left running.
+__global__ void wait_probe_kernel() {
+  __shared__ __align__(8) uint64_t bar;
+  const uint32_t b = stg::saddr(&bar);
+  if (threadIdx.x == 0) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(b));
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) wait_bounded(b, 0u);
+  __syncthreads();
+}
+#endif
+
 bool gemv_grouped_read_and_clear_timeout(cudaError_t* err) {
   unsigned int v = 0;
   const unsigned int zero = 0;
@@ -707,3 +788,11 @@ bool gemv_grouped_read_and_clear_timeout(cudaError_t* err) {
 }
 
 }  // namespace wq
+
+#ifdef WQ_TEST_HOOKS
+// Test builds only: launch the wait probe on `stream`; 0 on success.
+extern "C" int wq_test_expire_wait(void* stream) {
+  wq::wait_probe_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>();
+  return cudaGetLastError() == cudaSuccess ? 0 : 7;
+}
+#endif

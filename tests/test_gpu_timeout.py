@@ -1,12 +1,15 @@
 """Bounded device waits (failure handling without a GPU fault).
 
-libwq_shortwait.so is the library built with a pipeline-wait limit of 0, so
-every wait of the decode kernels that has not already completed gives up at
-once.  In a child process, the M = 1 GEMV, the 2..8-token warp-MMA GEMV and
-the grouped GEMV of that build must each report WQ_ERR_DEVICE_TIMEOUT through
-wq_last_device_error (their copies in flight are drained, so the context stays
-usable), and right after, in the same process, the normal library must compute
-y correctly and report no expired wait."""
+libwq_shortwait.so is the test build of the library: pipeline-wait limit 0 and
+one test hook, wq_test_expire_wait, a kernel whose bounded wait is on an
+mbarrier that nothing arrives on.  In a child process:
+  * the hook's wait runs out and wq_last_device_error reports
+    WQ_ERR_DEVICE_TIMEOUT once (a second read finds the flag cleared);
+  * the decode kernels of that build (M = 1 GEMV, 2..8-token warp-MMA GEMV,
+    grouped GEMV) run with a zero limit: each wait either finds its stage
+    landed or gives up, drains its copies and leaves;
+  * right after, in the same process and context, the normal library computes
+    y correctly and reports no expired wait."""
 from __future__ import annotations
 
 import ctypes
@@ -39,10 +42,15 @@ def _child(q):
         short.wq_gemm_grouped.argtypes = [ctypes.POINTER(wq.Linear), ci, i64, ci, vp, ctypes.c_size_t, vp]
         short.wq_gemm_grouped.restype = ci
         short.wq_last_device_error.restype = ci
+        short.wq_test_expire_wait.argtypes = [vp]
+        short.wq_test_expire_wait.restype = ci
+        res = {}
+        res["probe_launch"] = short.wq_test_expire_wait(None)
+        res["probe_status"] = short.wq_last_device_error()
+        res["probe_cleared"] = short.wq_last_device_error()
         N, K, bits, group = 96, 2048, 4, 128
         Wh = wq_inputs.weight_f16(60, 0, N, K)
         c, s, z = wq.wq_quantize_rtn(torch.from_numpy(Wh).cuda(), bits, group)
-        res = {}
         for M in (1, 4):
             x = wq_inputs.activations_bf16(60, M, M, K).cuda()
             y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
@@ -85,9 +93,12 @@ def test_expired_waits_are_reported_and_the_context_survives():
     p.join(timeout=60)
     assert kind == "ok", res
     assert p.exitcode == 0
+    assert res["probe_launch"] == 0, res
+    assert res["probe_status"] == 8, res                     # WQ_ERR_DEVICE_TIMEOUT
+    assert res["probe_cleared"] == 0, res
     for k in ("launch_M1", "launch_M4", "launch_grouped"):
-        assert res[k] == 0, (k, res)                       # the launches themselves succeed
+        assert res[k] == 0, (k, res)                         # the launches themselves succeed
     for k in ("timeout_M1", "timeout_M4", "timeout_grouped"):
-        assert res[k] == 8, (k, res)                       # WQ_ERR_DEVICE_TIMEOUT
+        assert res[k] in (0, 8), (k, res)                    # done, or gave up and reported it
     assert res["second_read_clears"] == 0
     assert res["normal_after"] == 0
