@@ -214,6 +214,31 @@ wq_status wq_gemm_grouped(const wq_linear* linears, int count, int64_t M, int bi
  * none is needed or an argument is invalid).  Needs no device. */
 size_t wq_gemm_grouped_workspace_size(const wq_linear* linears, int count, int64_t M, int bits);
 
+/*
+ * wq_gemm_grouped_noalloc -- wq_gemm_grouped for callers that cannot allocate
+ * device memory at the point of the call (a serving runtime that hands all
+ * GPU memory to its own pool at start-up, code running during CUDA graph
+ * capture, a real-time decode loop in which an allocation could synchronise
+ * the device or fail).  The pages have no counterpart: this is an interface
+ * convenience of this library, not a step of the method.
+ *
+ * Same arguments, checks, kernels and results as wq_gemm_grouped, without the
+ * workspace: the library keeps one built-in workspace of 8 MiB per GPU (a
+ * device array that every GPU loading the library holds until the process
+ * exits).  A call whose linears need more than 8 MiB of workspace (see
+ * wq_gemm_grouped_workspace_size) returns WQ_ERR_WORKSPACE before anything
+ * is launched.  The call allocates and frees nothing; each call clears the
+ * workspace's tile counters on `stream` before its kernels run.
+ *   - The first call on a device looks up the array's device address (and
+ *     sets the kernels' attributes); make that first call before any stream
+ *     capture.
+ *   - All calls on a device share the one array and it keeps the last call's
+ *     contents: calls whose kernels overlap on the GPU (different streams
+ *     without ordering, or several host threads) race and give wrong results.
+ *     Order them on one stream.
+ */
+wq_status wq_gemm_grouped_noalloc(const wq_linear* linears, int count, int64_t M, int bits, void* stream);
+
 /* Number of uint32 words of packed codes for an [N, K] matrix: N*K*bits/32
  * (0 if bits or K are invalid). */
 size_t wq_codes_words(int64_t N, int64_t K, int bits);

@@ -34,6 +34,7 @@ WQ_ERR_WORKSPACE = 9
 
 # Functions the header declares (the tests check the library exports them).
 EXPORTED = ("wq_quantize_rtn", "wq_quantize_rtn_sym", "wq_gemm", "wq_gemm_grouped", "wq_gemm_grouped_workspace_size",
+            "wq_gemm_grouped_noalloc",
             "wq_codes_words", "wq_params_count", "wq_status_string", "wq_last_device_error")
 
 
@@ -60,6 +61,8 @@ def _load():
     lp = ctypes.POINTER(Linear)
     lib.wq_gemm_grouped.argtypes = [lp, ci, i64, ci, vp, ctypes.c_size_t, vp]
     lib.wq_gemm_grouped.restype = ci
+    lib.wq_gemm_grouped_noalloc.argtypes = [lp, ci, i64, ci, vp]
+    lib.wq_gemm_grouped_noalloc.restype = ci
     lib.wq_gemm_grouped_workspace_size.argtypes = [lp, ci, i64, ci]
     lib.wq_gemm_grouped_workspace_size.restype = ctypes.c_size_t
     lib.wq_codes_words.argtypes = [i64, i64, ci]
@@ -222,4 +225,20 @@ def wq_gemm_grouped(items, bits: int, workspace=None, stream=None):
     st = lib.wq_gemm_grouped(arr, len(items), M, bits, _ptr(workspace),
                              workspace.numel() * workspace.element_size(), _stream_ptr(stream))
     _check(st, "wq_gemm_grouped")
+    return ys
+
+
+def wq_gemm_grouped_noalloc(items, bits: int, stream=None):
+    """``wq_gemm_grouped`` on the library's built-in 8 MiB workspace, for
+    callers that cannot allocate device memory when they call.  Every item
+    must carry its output ``y`` (x, codes, scales, zeros, N, K, group, y):
+    nothing is allocated here either."""
+    if not items:
+        return []
+    if any(len(it) < 8 or it[7] is None for it in items):
+        raise ValueError("wq_gemm_grouped_noalloc allocates nothing: pass every y")
+    M = items[0][0].shape[0]
+    arr, ys = _linear_array(items, M)
+    st = lib.wq_gemm_grouped_noalloc(arr, len(items), M, bits, _stream_ptr(stream))
+    _check(st, "wq_gemm_grouped_noalloc")
     return ys

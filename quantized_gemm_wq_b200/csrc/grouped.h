@@ -81,4 +81,9 @@ cudaError_t launch_gemv_grouped(const GroupedLinear* lins, int count, int M, int
                                 cudaStream_t st);
 bool gemv_grouped_read_and_clear_timeout(cudaError_t* err);
 
+// The built-in workspace of wq_gemm_grouped_noalloc (noalloc.cu): its size,
+// and its device address on the current device (looked up on first use).
+size_t static_workspace_bytes();
+cudaError_t static_workspace(void** addr);
+
 }  // namespace wq

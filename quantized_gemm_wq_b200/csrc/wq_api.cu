@@ -223,6 +223,41 @@ wq_status wq_gemm_grouped(const wq_linear* linears, int count, int64_t M, int bi
   return e == cudaSuccess ? WQ_OK : WQ_ERR_CUDA;
 }
 
+wq_status wq_gemm_grouped_noalloc(const wq_linear* linears, int count, int64_t M, int bits, void* stream) {
+  if (!linears) return WQ_ERR_NULL;
+  if (count < 1) return WQ_ERR_SHAPE;
+  if (!valid_bits(bits)) return WQ_ERR_BITS;
+  for (int i = 0; i < count; ++i) {
+    const wq_status st = check_linear(linears[i], M, bits);
+    if (st != WQ_OK) return st;
+  }
+  const std::vector<wq::GroupedLinear> fast = grouped_fast_list(linears, count, M);
+  const size_t need =
+      fast.empty() ? 0 : wq::grouped_workspace_layout(fast.data(), int(fast.size()), int(M), 0, nullptr);
+  if (need > wq::static_workspace_bytes()) return WQ_ERR_WORKSPACE;
+  wq_status st = check_device();
+  if (st != WQ_OK) return st;
+  const auto strm = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaSuccess;
+  if (!fast.empty()) {
+    void* base = nullptr;
+    e = wq::static_workspace(&base);
+    if (e != cudaSuccess) return WQ_ERR_CUDA;
+    wq::WsLayout ws;
+    wq::grouped_workspace_layout(fast.data(), int(fast.size()), int(M), reinterpret_cast<uintptr_t>(base), &ws);
+    // Every call shares the array: the tile counters must start at zero, and a
+    // call that gave up a bounded wait may have left some set.
+    e = cudaMemsetAsync(ws.cnt, 0, sizeof(unsigned) * wq::kMaxCtas, strm);
+    if (e == cudaSuccess) e = wq::launch_gemv_grouped(fast.data(), int(fast.size()), int(M), bits, ws, strm);
+  }
+  for (int i = 0; i < count && e == cudaSuccess; ++i) {
+    const wq::GroupedLinear g = to_grouped(linears[i]);
+    if (M <= wq::kGemvMaxM && wq::grouped_supported(g.K, g.group)) continue;
+    e = dispatch_one(g.x, M, g.N, g.K, g.codes, g.scales, g.zeros, bits, g.group, g.y, strm);
+  }
+  return e == cudaSuccess ? WQ_OK : WQ_ERR_CUDA;
+}
+
 wq_status wq_last_device_error(void) {
   cudaError_t e[5] = {cudaSuccess, cudaSuccess, cudaSuccess, cudaSuccess, cudaSuccess};
   const bool hit = wq::gemm_tc_read_and_clear_timeout(&e[0]) | wq::gemv_m1_tma_read_and_clear_timeout(&e[1]) |
