@@ -99,6 +99,16 @@ __device__ __forceinline__ void mma_bf16(float (&c)[4], uint32_t a0, uint32_t a1
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// The same MMA with a zero accumulator input: D = A B.
+__device__ __forceinline__ void mma_bf16_z(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                           uint32_t b0, uint32_t b1) {
+  const float z = 0.0f;
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%10, %10, %10, %10};"
+      : "=f"(c[0]), "=f"(c[1]), "=f"(c[2]), "=f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(z));
+}
+
 // Accumulators of a lane for one quad: [tile][chain][4], tile 0 the rows of
 // the lane's first A fragment pair (words w[0], w[1]), tile 1 the next
 // (w[2], w[3]); chain J % 2, so consecutive MMAs of a tile do not wait for
@@ -109,17 +119,23 @@ struct QuadAcc {
 
 // MMA J..7 of 16-row tile T over a quad (A rows from the words wa, wb)
 // against one 8-token B operand (xb); with TWO the same A fragments also meet
-// the second 8-token operand (xb2).
-template <int BITS, int T, int J, bool TWO>
+// the second 8-token operand (xb2).  FRESH: the first MMA of each chain
+// starts from zero instead of adding to the accumulators.
+template <int BITS, int T, int J, bool TWO, bool FRESH>
 struct QuadMma {
   __device__ __forceinline__ static void run(QuadAcc& a, QuadAcc& a2, const uint32_t (&wa)[BITS],
                                              const uint32_t (&wb)[BITS], const uint32_t (&xb)[16],
                                              const uint32_t (&xb2)[16]) {
     const uint32_t a0 = unit_pair<BITS, 2 * J>(wa), a1 = unit_pair<BITS, 2 * J>(wb);
     const uint32_t a2r = unit_pair<BITS, 2 * J + 1>(wa), a3 = unit_pair<BITS, 2 * J + 1>(wb);
-    mma_bf16(a.c[T][J & 1], a0, a1, a2r, a3, xb[2 * J], xb[2 * J + 1]);
-    if constexpr (TWO) mma_bf16(a2.c[T][J & 1], a0, a1, a2r, a3, xb2[2 * J], xb2[2 * J + 1]);
-    if constexpr (J + 1 < 8) QuadMma<BITS, T, J + 1, TWO>::run(a, a2, wa, wb, xb, xb2);
+    if constexpr (FRESH && J < 2) {
+      mma_bf16_z(a.c[T][J & 1], a0, a1, a2r, a3, xb[2 * J], xb[2 * J + 1]);
+      if constexpr (TWO) mma_bf16_z(a2.c[T][J & 1], a0, a1, a2r, a3, xb2[2 * J], xb2[2 * J + 1]);
+    } else {
+      mma_bf16(a.c[T][J & 1], a0, a1, a2r, a3, xb[2 * J], xb[2 * J + 1]);
+      if constexpr (TWO) mma_bf16(a2.c[T][J & 1], a0, a1, a2r, a3, xb2[2 * J], xb2[2 * J + 1]);
+    }
+    if constexpr (J + 1 < 8) QuadMma<BITS, T, J + 1, TWO, FRESH>::run(a, a2, wa, wb, xb, xb2);
   }
 };
 
@@ -144,6 +160,11 @@ struct LinRegs {
   int64_t stage0;
   int N, K, G, TS, tiles;
   FastDiv upg;
+  // Groups that tile a 1024-code stage (g = 128, 256, 512, 1024): a warp's
+  // quad of every stage is in a new group, the group's index in the stage is
+  // warp >> qshift, the stage's first group is 8 t >> qshift.
+  bool tiles_stage;
+  int qshift;
   __device__ __forceinline__ void load(const GLin& L) {
     scales = L.scales;
     zeros = L.zeros;
@@ -157,6 +178,9 @@ struct LinRegs {
     TS = L.TS;
     tiles = L.tiles;
     upg = L.upg;
+    const int qpg = int(upg.d) >> 2;        // 128-code quads per group
+    tiles_stage = qpg <= 8 && (8 % qpg) == 0;
+    qshift = qpg >= 8 ? 3 : (qpg >= 4 ? 2 : (qpg >= 2 ? 1 : 0));
   }
 };
 
@@ -191,7 +215,8 @@ __host__ __device__ constexpr int xp_chunk_pos(int c) { return (c & ~7) | ((c ^ 
 template <int MT>
 struct Tok {
   static constexpr int SXW = MT < 4 ? 4 : MT;     // floats of sum x per quad (16-byte multiple)
-  static constexpr int NC = MT == 16 ? 4 : 2;     // accumulator columns per lane
+  // accumulator columns per lane (column 2 tq + 1 never holds a token when MT = 1)
+  static constexpr int NC = MT == 16 ? 4 : (MT == 1 ? 1 : 2);
 };
 
 // ---------------------------------------------------------------------------
@@ -410,6 +435,11 @@ __global__ void __launch_bounds__(kThreads, MINB) gemv_grouped_kernel(const __gr
   int rw[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) rw[i] = mma_row<BITS>(g) + 8 * i;
+  // With one or two tokens only the lanes t = 0 hold real accumulator
+  // columns; the fold then moves each row's dot product to a lane of its own
+  // (lane l: MMA row l % 8 of quarter l / 8, i.e. weight row lrow).
+  constexpr bool LR = MT <= 2;
+  const int lrow = mma_row<BITS>(lane & 7) + 8 * (lane >> 3);
   uint32_t uoff[4][unit_pieces<BITS>()];
 #pragma unroll
   for (int i = 0; i < 4; ++i) unit_offsets<BITS>(rw[i], 4 * warp + tq, uoff[i]);
@@ -480,34 +510,41 @@ __global__ void __launch_bounds__(kThreads, MINB) gemv_grouped_kernel(const __gr
       }
       // sum x of the quad for this lane's tokens
       const float* sxq = reinterpret_cast<const float*>(smem + C::OFF_SX + s * C::SXB) + warp * SXW;
+      if constexpr (LR) {
 #pragma unroll
-      for (int c = 0; c < NC; ++c)
-        if (tok_of(c) < MT) sxg[c] += sxq[tok_of(c)];
+        for (int c = 0; c < MT; ++c) sxg[c] += sxq[c];
+      } else {
+#pragma unroll
+        for (int c = 0; c < NC; ++c)
+          if (tok_of(c) < MT) sxg[c] += sxq[tok_of(c)];
+      }
       const uint32_t stage = ring + uint32_t(s * C::SB);
-      {
-        uint32_t wa[BITS], wb[BITS];
-        load_unit_at<BITS>(stage, uoff[0], wa);
-        load_unit_at<BITS>(stage, uoff[1], wb);
-        QuadMma<BITS, 0, 0, MT == 16>::run(qa, qa2, wa, wb, xa, xb2);
-      }
-      {
-        uint32_t wa[BITS], wb[BITS];
-        load_unit_at<BITS>(stage, uoff[2], wa);
-        load_unit_at<BITS>(stage, uoff[3], wb);
-        QuadMma<BITS, 1, 0, MT == 16>::run(qa, qa2, wa, wb, xa, xb2);
-      }
-      // fold into y when the next quad of this warp is in another group, or absent
-      const uint32_t uq = uint32_t(kq / 32);
-      const int gq = int(L.upg.div(uq));
-      const bool next_in = !seg_end && kq + 1024 < L.K;
-      if (!next_in || int(L.upg.div(uq + 32)) != gq) {
-        // (s, z) of row rw[r]: half (e0 & 1) + rel of the row's window, e0 =
-        // n G + gfirst its first needed half (see the producer)
-        const int gfirst = int(L.upg.div(uint32_t(q.t) * 32));
-        const int rel = gq - gfirst;
+      // Fold the quad's dot products D into y: acc += s (D 2^69 - z sum x),
+      // (s, z) of row rw[r] at half h(r) of the row's window in the slot.
+      auto fold = [&](int gfirst, int rel) {
         const __half* szs = reinterpret_cast<const __half*>(smem + C::OFF_SZ + s * C::SZB);
         // e0 = n G + gfirst has the parity of gfirst, plus that of n when G is odd
         const int gpar = L.G & 1;
+        if constexpr (LR) {
+          // lane l takes row lrow: quarter r = l / 8 of lane 4 (l % 8)'s rows
+          const int h = ((gpar * (int(q.r) * 32 + lrow) + gfirst) & 1) + rel;
+          const __half* rs = szs + lrow * (2 * kSzRow);
+          const float sc = __half2float(rs[h]);
+          const float zr = __half2float(L.zeros ? rs[2 * kSzW + h] : hz);
+          const int src = 4 * (lane & 7), rq = lane >> 3;
+#pragma unroll
+          for (int c = 0; c < MT; ++c) {
+            float mine = 0.0f;
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+              const int t = r >> 1, ce = 2 * (r & 1) + c;
+              const float d = __shfl_sync(0xffffffffu, qa.c[t][0][ce] + qa.c[t][1][ce], src);
+              mine = rq == r ? d : mine;
+            }
+            acc[0][c] = fmaf(sc, fmaf(mine, 0x1p69f, -zr * sxg[c]), acc[0][c]);
+          }
+          return;
+        }
         float2 zs[4];
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
@@ -528,7 +565,47 @@ __global__ void __launch_bounds__(kThreads, MINB) gemv_grouped_kernel(const __gr
             acc[r][c] = fmaf(zs[r].x, fmaf(d, 0x1p69f, -zs[r].y * sxg[c]), acc[r][c]);
           }
         }
-        zero_quad();
+      };
+      if (L.tiles_stage) {
+        // every quad is a group of its own (or part of one inside this
+        // stage): MMAs start from zero, the fold follows at once
+        {
+          uint32_t wa[BITS], wb[BITS];
+          load_unit_at<BITS>(stage, uoff[0], wa);
+          load_unit_at<BITS>(stage, uoff[1], wb);
+          QuadMma<BITS, 0, 0, MT == 16, true>::run(qa, qa2, wa, wb, xa, xb2);
+        }
+        {
+          uint32_t wa[BITS], wb[BITS];
+          load_unit_at<BITS>(stage, uoff[2], wa);
+          load_unit_at<BITS>(stage, uoff[3], wb);
+          QuadMma<BITS, 1, 0, MT == 16, true>::run(qa, qa2, wa, wb, xa, xb2);
+        }
+        fold((q.t * 8) >> L.qshift, warp >> L.qshift);
+#pragma unroll
+        for (int c = 0; c < NC; ++c) sxg[c] = 0.0f;
+      } else {
+        {
+          uint32_t wa[BITS], wb[BITS];
+          load_unit_at<BITS>(stage, uoff[0], wa);
+          load_unit_at<BITS>(stage, uoff[1], wb);
+          QuadMma<BITS, 0, 0, MT == 16, false>::run(qa, qa2, wa, wb, xa, xb2);
+        }
+        {
+          uint32_t wa[BITS], wb[BITS];
+          load_unit_at<BITS>(stage, uoff[2], wa);
+          load_unit_at<BITS>(stage, uoff[3], wb);
+          QuadMma<BITS, 1, 0, MT == 16, false>::run(qa, qa2, wa, wb, xa, xb2);
+        }
+        // fold when the next quad of this warp is in another group, or absent
+        const uint32_t uq = uint32_t(kq / 32);
+        const int gq = int(L.upg.div(uq));
+        const bool next_in = !seg_end && kq + 1024 < L.K;
+        if (!next_in || int(L.upg.div(uq + 32)) != gq) {
+          const int gfirst = int(L.upg.div(uint32_t(q.t) * 32));
+          fold(gfirst, gq - gfirst);
+          zero_quad();
+        }
       }
     }
     __syncwarp();
@@ -537,19 +614,26 @@ __global__ void __launch_bounds__(kThreads, MINB) gemv_grouped_kernel(const __gr
     if (seg_end) {
       // ---------------------------------------------------- tile epilogue
       float* rb = red + (C::RB == 2 ? (tcount & 1) : 0) * (kNW * MT * 32);
+      if constexpr (LR) {
 #pragma unroll
-      for (int c = 0; c < NC; ++c)
-        if (tok_of(c) < MT) {
+        for (int c = 0; c < MT; ++c) rb[(warp * MT + c) * 32 + lrow] = acc[0][c];
+      } else {
 #pragma unroll
-          for (int r = 0; r < 4; ++r) rb[(warp * MT + tok_of(c)) * 32 + rw[r]] = acc[r][c];
-        }
+        for (int c = 0; c < NC; ++c)
+          if (tok_of(c) < MT) {
+#pragma unroll
+            for (int r = 0; r < 4; ++r) rb[(warp * MT + tok_of(c)) * 32 + rw[r]] = acc[r][c];
+          }
+      }
       asm volatile("bar.sync 1, %0;" ::"n"(32 * kNW) : "memory");
       const int64_t tb = L.stage0 + q.r * L.TS, te = tb + L.TS;
       const bool whole = seg_start <= tb && te <= se;
       const int64_t row0 = q.r * 32;
       // parked partials: slot 0 for a CTA's first tile, slot 1 for its last
       const int myslot = sb >= tb ? 0 : 1;
-      for (int idx = tid; idx < 32 * MT; idx += 32 * kNW) {
+      // the summing threads rotate over the warps from tile to tile
+      const int rt = (tid + 32 * (tcount & 7)) & (32 * kNW - 1);
+      for (int idx = rt; idx < 32 * MT; idx += 32 * kNW) {
         const int m = idx >> 5, row = idx & 31;
         float v = 0.0f;
 #pragma unroll
@@ -591,12 +675,16 @@ __global__ void __launch_bounds__(kThreads, MINB) gemv_grouped_kernel(const __gr
         for (int c = 0; c < NC; ++c) acc[r][c] = 0.0f;
       seg_start = sb + i + 1;
     }
-    // next stage; a new linear's fields are read once
+    // next stage; a new linear's fields are read once, and its first
+    // accumulating MMA must not add to what a fresh-start linear left behind
     if (++q.t == L.TS) {
       q.t = 0;
       if (++q.r == L.tiles) {
         q.r = 0;
-        if (++q.l < p.nlin && i + 1 < T) L.load(p.lin[q.l]);
+        if (++q.l < p.nlin && i + 1 < T) {
+          L.load(p.lin[q.l]);
+          zero_quad();
+        }
       }
     }
   }
@@ -618,16 +706,24 @@ int device_sms(int dev) {
   return v;
 }
 
-// Ring depth and resident CTAs per SM by token tile.
-template <int MT>
+// Ring depth and resident CTAs per SM: as many stages as the shared memory
+// of two CTAs per SM holds (one CTA for 16 tokens), because the achieved
+// bandwidth follows the bytes each SM keeps in flight.
+template <int BITS, int MT>
 struct Shape {
-  static constexpr int D = MT <= 4 ? 4 : (MT == 8 ? 3 : 2);
-  static constexpr int MINB = MT <= 8 ? 2 : 1;
+  static constexpr int kPer = BITS * 4096 + MT * 2048 + 8 * Tok<MT>::SXW * 4 + 32 * kSzRow * 4 + 16;
+  static constexpr int kRed = (MT <= 8 ? 2 : 1) * kNW * MT * 32 * 4;
+  static constexpr int kFixed = kRed + 64 + 16 + 1024;
+  // two CTAs per SM when two stages each still fit in half the shared memory
+  static constexpr int MINB = (MT <= 8 && 2 * kPer + kFixed <= 113 * 1024) ? 2 : 1;
+  static constexpr int kFit = ((MINB == 2 ? 113 : 226) * 1024 - kFixed) / kPer;
+  static constexpr int D = kFit < 2 ? 2 : (kFit > 12 ? 12 : kFit);
 };
 
 template <int BITS, int MT>
 cudaError_t launch_mt(const GroupedLinear* lins, int count, int M, const WsLayout& ws, cudaStream_t st) {
-  constexpr int D = Shape<MT>::D, MINB = Shape<MT>::MINB;
+  constexpr int D = Shape<BITS, MT>::D, MINB = Shape<BITS, MT>::MINB;
+  static_assert(GCfg<BITS, MT, D>::BYTES <= (MINB == 2 ? 113 : 226) * 1024, "shared memory");
   using C = GCfg<BITS, MT, D>;
   auto kern = gemv_grouped_kernel<BITS, MT, D, MINB>;
   int dev = 0;
