@@ -264,7 +264,9 @@ struct GCfg {
   static constexpr int XB = MT * 2048;                    // x': 8 quads x MT tokens x 256 B
   static constexpr int SXB = 8 * Tok<MT>::SXW * 4;        // sums per quad and token
   static constexpr int SZB = 32 * kSzRow * 4;             // raw (s, z) of 32 rows x up to 8 groups
-  static constexpr int RB = MT <= 8 ? 2 : 1;              // tile reduction buffers
+  // tile reduction buffers: with one or two tokens the warps meet through a
+  // per-buffer counter instead of a barrier, and a warp may run D tiles ahead
+  static constexpr int RB = MT <= 2 ? D + 1 : (MT <= 8 ? 2 : 1);
   static constexpr int REDB = RB * kNW * MT * 32 * 4;
   static constexpr int OFF_XP = D * SB;
   static constexpr int OFF_SX = OFF_XP + D * XB;
@@ -273,7 +275,8 @@ struct GCfg {
   static constexpr int OFF_ZERO = OFF_RED + REDB;         // 64 zero bytes: B of empty token columns
   static constexpr int OFF_BAR = OFF_ZERO + 64;           // full[D], empty[D]
   static constexpr int OFF_FLAG = OFF_BAR + 16 * D;
-  static constexpr int BYTES = OFF_FLAG + 16 + 1024;      // + alignment slack
+  static constexpr int OFF_TCNT = OFF_FLAG + 16;           // arrivals per reduction buffer
+  static constexpr int BYTES = OFF_TCNT + 4 * RB + 1024;   // + alignment slack
 };
 
 // Position in a CTA's stage range: linear l, row tile r, stage t of the tile.
@@ -319,6 +322,7 @@ __global__ void __launch_bounds__(kThreads, MINB) gemv_grouped_kernel(const __gr
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (threadIdx.x < 16) reinterpret_cast<uint32_t*>(smem + C::OFF_ZERO)[threadIdx.x] = 0u;
+  if (threadIdx.x < C::RB) reinterpret_cast<unsigned*>(smem + C::OFF_TCNT)[threadIdx.x] = 0u;
   __syncthreads();
   if (T <= 0) return;
 
@@ -613,24 +617,72 @@ __global__ void __launch_bounds__(kThreads, MINB) gemv_grouped_kernel(const __gr
 
     if (seg_end) {
       // ---------------------------------------------------- tile epilogue
-      float* rb = red + (C::RB == 2 ? (tcount & 1) : 0) * (kNW * MT * 32);
-      if constexpr (LR) {
-#pragma unroll
-        for (int c = 0; c < MT; ++c) rb[(warp * MT + c) * 32 + lrow] = acc[0][c];
-      } else {
-#pragma unroll
-        for (int c = 0; c < NC; ++c)
-          if (tok_of(c) < MT) {
-#pragma unroll
-            for (int r = 0; r < 4; ++r) rb[(warp * MT + tok_of(c)) * 32 + rw[r]] = acc[r][c];
-          }
-      }
-      asm volatile("bar.sync 1, %0;" ::"n"(32 * kNW) : "memory");
       const int64_t tb = L.stage0 + q.r * L.TS, te = tb + L.TS;
       const bool whole = seg_start <= tb && te <= se;
       const int64_t row0 = q.r * 32;
       // parked partials: slot 0 for a CTA's first tile, slot 1 for its last
       const int myslot = sb >= tb ? 0 : 1;
+      // contributors of a cut tile: the CTAs whose ranges hold its first and last stage
+      const int64_t ca = ((tb + 1) * p.P - 1) / p.total, cbk = (te * p.P - 1) / p.total;
+      if constexpr (LR) {
+        // Each warp parks its 32 row sums; the last warp to arrive on the
+        // buffer's counter adds the eight in warp order and writes y (or the
+        // CTA's partial of a cut tile).  No barrier: the others go on.
+        const int slot = tcount % C::RB;
+        float* rb = red + slot * (kNW * MT * 32);
+        unsigned* tcnt = reinterpret_cast<unsigned*>(smem + C::OFF_TCNT) + slot;
+#pragma unroll
+        for (int c = 0; c < MT; ++c) rb[(warp * MT + c) * 32 + lrow] = acc[0][c];
+        __syncwarp();
+        unsigned arrived = 0;
+        if (lane == 0) {
+          __threadfence_block();
+          arrived = atomicAdd(tcnt, 1u);
+        }
+        if (__shfl_sync(0xffffffffu, arrived, 0) == unsigned(kNW - 1)) {
+          __threadfence_block();
+#pragma unroll
+          for (int m = 0; m < MT; ++m) {
+            float v = 0.0f;
+#pragma unroll
+            for (int wv = 0; wv < kNW; ++wv) v += rb[(wv * MT + m) * 32 + lane];
+            if (whole) {
+              if (m < p.M && row0 + lane < L.N) L.y[int64_t(m) * L.N + row0 + lane] = __float2bfloat16_rn(v);
+            } else {
+              p.part[((cta * 2 + myslot) * MT + m) * 32 + lane] = v;
+            }
+          }
+          if (!whole) {
+            __threadfence();
+            __syncwarp();
+            unsigned old = 0;
+            if (lane == 0) old = atomicAdd(p.cnt + ca, 1u);
+            if (__shfl_sync(0xffffffffu, old, 0) == unsigned(cbk - ca)) {
+              __threadfence();
+              const int slot_a = range_start(p, ca) < tb ? 1 : 0;
+#pragma unroll
+              for (int m = 0; m < MT; ++m) {
+                float v = 0.0f;
+                for (int64_t cc = ca; cc <= cbk; ++cc)
+                  v += __ldcg(p.part + ((cc * 2 + (cc == ca ? slot_a : 0)) * MT + m) * 32 + lane);
+                if (m < p.M && row0 + lane < L.N) L.y[int64_t(m) * L.N + row0 + lane] = __float2bfloat16_rn(v);
+              }
+              __syncwarp();
+              if (lane == 0) atomicExch(p.cnt + ca, 0u);
+            }
+          }
+          __syncwarp();
+          if (lane == 0) atomicExch(tcnt, 0u);     // the buffer is free again
+        }
+      } else {
+      float* rb = red + (C::RB == 2 ? (tcount & 1) : 0) * (kNW * MT * 32);
+#pragma unroll
+      for (int c = 0; c < NC; ++c)
+        if (tok_of(c) < MT) {
+#pragma unroll
+          for (int r = 0; r < 4; ++r) rb[(warp * MT + tok_of(c)) * 32 + rw[r]] = acc[r][c];
+        }
+      asm volatile("bar.sync 1, %0;" ::"n"(32 * kNW) : "memory");
       // the summing threads rotate over the warps from tile to tile
       const int rt = (tid + 32 * (tcount & 7)) & (32 * kNW - 1);
       for (int idx = rt; idx < 32 * MT; idx += 32 * kNW) {
@@ -645,8 +697,6 @@ __global__ void __launch_bounds__(kThreads, MINB) gemv_grouped_kernel(const __gr
         }
       }
       if (!whole) {
-        // contributors: the CTAs whose ranges hold the tile's first and last stage
-        const int64_t ca = ((tb + 1) * p.P - 1) / p.total, cbk = (te * p.P - 1) / p.total;
         __threadfence();
         asm volatile("bar.sync 1, %0;" ::"n"(32 * kNW) : "memory");
         if (tid == 0) {
@@ -668,6 +718,7 @@ __global__ void __launch_bounds__(kThreads, MINB) gemv_grouped_kernel(const __gr
         }
       }
       if constexpr (C::RB == 1) asm volatile("bar.sync 1, %0;" ::"n"(32 * kNW) : "memory");
+      }
       ++tcount;
 #pragma unroll
       for (int r = 0; r < 4; ++r)
@@ -711,9 +762,11 @@ int device_sms(int dev) {
 // bandwidth follows the bytes each SM keeps in flight.
 template <int BITS, int MT>
 struct Shape {
-  static constexpr int kPer = BITS * 4096 + MT * 2048 + 8 * Tok<MT>::SXW * 4 + 32 * kSzRow * 4 + 16;
-  static constexpr int kRed = (MT <= 8 ? 2 : 1) * kNW * MT * 32 * 4;
-  static constexpr int kFixed = kRed + 64 + 16 + 1024;
+  // per stage: codes, x', sums, (s, z), barriers (and a reduction buffer with <= 2 tokens)
+  static constexpr int kPer = BITS * 4096 + MT * 2048 + 8 * Tok<MT>::SXW * 4 + 32 * kSzRow * 4 + 16 +
+                              (MT <= 2 ? kNW * MT * 32 * 4 + 4 : 0);
+  static constexpr int kRed = (MT <= 2 ? 1 : (MT <= 8 ? 2 : 1)) * kNW * MT * 32 * 4;
+  static constexpr int kFixed = kRed + 64 + 16 + 64 + 1024;
   // two CTAs per SM when two stages each still fit in half the shared memory
   static constexpr int MINB = (MT <= 8 && 2 * kPer + kFixed <= 113 * 1024) ? 2 : 1;
   static constexpr int kFit = ((MINB == 2 ? 113 : 226) * 1024 - kFixed) / kPer;
