@@ -53,7 +53,9 @@ cudaError_t dispatch_one(const __nv_bfloat16* x, int64_t M, int64_t N, int64_t K
                          const __half* s, const __half* z, int bits, int64_t g, __nv_bfloat16* y,
                          cudaStream_t strm) {
   cudaError_t e;
-  if (M > wq::kGemvMaxM && wq::gemm_tc_supported(K, bits)) {
+  if (M > wq::kGemvMaxM && wq::gemm_sw_supported(M, K)) {
+    e = wq::launch_gemm_sw(x, M, N, K, codes, s, z, bits, g, y, strm);
+  } else if (M > wq::kGemvMaxM && wq::gemm_tc_supported(K, bits)) {
     e = wq::launch_gemm_tc(x, M, N, K, codes, s, z, bits, g, y, strm);
   } else {
     // Small batches, and K that the tensor-core GEMM cannot stage with TMA
@@ -259,10 +261,10 @@ wq_status wq_gemm_grouped_noalloc(const wq_linear* linears, int count, int64_t M
 }
 
 wq_status wq_last_device_error(void) {
-  cudaError_t e[5] = {cudaSuccess, cudaSuccess, cudaSuccess, cudaSuccess, cudaSuccess};
+  cudaError_t e[6] = {cudaSuccess, cudaSuccess, cudaSuccess, cudaSuccess, cudaSuccess, cudaSuccess};
   const bool hit = wq::gemm_tc_read_and_clear_timeout(&e[0]) | wq::gemv_m1_tma_read_and_clear_timeout(&e[1]) |
                    wq::gemv_tc_read_and_clear_timeout(&e[2]) | wq::gemv_mma_read_and_clear_timeout(&e[3]) |
-                   wq::gemv_grouped_read_and_clear_timeout(&e[4]);
+                   wq::gemv_grouped_read_and_clear_timeout(&e[4]) | wq::gemm_sw_read_and_clear_timeout(&e[5]);
   for (cudaError_t x : e)
     if (x != cudaSuccess) return WQ_ERR_CUDA;
   return hit ? WQ_ERR_DEVICE_TIMEOUT : WQ_OK;

@@ -93,6 +93,14 @@ bool gemv_mma_read_and_clear_timeout(cudaError_t* err);
 // True when the tensor-core path can stage this K with TMA (K a multiple of 128).
 bool gemm_tc_supported(int64_t K, int bits);
 
+// Batches of 17..255 rows on the tensor cores with the weight rows on the
+// MMA's M side (gemm_sw.cu); K a multiple of 128.
+bool gemm_sw_supported(int64_t M, int64_t K);
+cudaError_t launch_gemm_sw(const __nv_bfloat16* x, int64_t M, int64_t N, int64_t K, const uint32_t* codes,
+                           const __half* scales, const __half* zeros, int bits, int64_t g, __nv_bfloat16* y,
+                           cudaStream_t st);
+bool gemm_sw_read_and_clear_timeout(cudaError_t* err);
+
 cudaError_t launch_gemm_tc(const __nv_bfloat16* x, int64_t M, int64_t N, int64_t K,
                            const uint32_t* codes, const __half* scales, const __half* zeros,
                            int bits, int64_t g, __nv_bfloat16* y, cudaStream_t st);
