@@ -340,7 +340,7 @@ def leg_stack(args, seed, sampler, world):
             del ws
         else:
             t = reduce_max(graph_time([per_linear_fn(items, bits)], n, args.warmup, sampler))
-            path = "wq_gemm per linear (tcgen05 GEMM)"
+            path = "wq_gemm per linear (swap-AB tcgen05 GEMM)"
         other[str(M)] = {"us_per_step": t * 1e3, "GBps": world * gbps(step_bytes(HEADLINE, M), t),
                          "TFLOPs": world * step_flops(HEADLINE, M) / (t * 1e-3) / 1e12, "path": path}
         del items
@@ -616,8 +616,9 @@ def main(argv=None):
 
 def run_case(case: str) -> None:
     """One small profiling case (for ncu), after 3 untimed repetitions:
-    ``stack:<M>:<layers>`` one grouped decode step over the first <layers>
-    layers of the 32-layer stack (layers >= 2 exceed L2); ``gemv:<i>`` /
+    ``stack:<M>:<layers>`` one decode step over the first <layers> layers of
+    the 32-layer stack (layers >= 2 exceed L2): one wq_gemm_grouped call for
+    M <= 16, one wq_gemm per linear above; ``gemv:<i>`` /
     ``gemv16:<i>`` one wq_gemm of projection i of the 3-bit layer at M = 1 / 16;
     ``prefill:<i>`` one prefill GEMM (M = 2048) of the 13B-shaped workload."""
     import torch
@@ -633,9 +634,13 @@ def run_case(case: str) -> None:
             c, s, z = wq.wq_quantize_rtn(W, w["bits"], w["group"])
             del W
             items.append((device_x(0, li, M, K), c, s, z, N, K, w["group"]))
-        ws = wq.grouped_workspace(items, w["bits"])
+        ws = wq.grouped_workspace(items, w["bits"]) if M <= 16 else None
         for _ in range(4):
-            wq.wq_gemm_grouped(items, w["bits"], workspace=ws)
+            if M <= 16:
+                wq.wq_gemm_grouped(items, w["bits"], workspace=ws)
+            else:
+                for (x, c, s, z, N, K, g) in items:
+                    wq.wq_gemm(x, c, s, z, w["bits"], g, N, K)
         torch.cuda.synchronize()
         assert wq.wq_last_device_error() == wq.WQ_OK
         print(json.dumps({"case": case, "linears": len(items), "ok": True}))
