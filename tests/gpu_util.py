@@ -41,6 +41,11 @@ def oracle_quantize(Wh: np.ndarray, bits: int, group: int):
     return oracle.pack(q, bits), s, z
 
 
+# Largest max |y - y_ref| / sum_k |x w'| seen by assert_y_close in this run,
+# with the check that produced it (printed in the pytest summary).
+WORST = {"ratio": 0.0, "what": ""}
+
+
 def assert_y_close(y_gpu: np.ndarray, y_ref: np.ndarray, bound: np.ndarray, what: str = ""):
     err = np.abs(y_gpu.astype(np.float64) - y_ref)
     lim = REL_TOL * bound + OUT_ROUND * np.abs(y_ref) + ABS_TOL
@@ -50,7 +55,10 @@ def assert_y_close(y_gpu: np.ndarray, y_ref: np.ndarray, bound: np.ndarray, what
         raise AssertionError(f"{what}: {int(bad.sum())} of {bad.size} outside tolerance; first "
                              f"{tuple(i)} gpu={y_gpu[tuple(i)]} ref={y_ref[tuple(i)]} "
                              f"bound={bound[tuple(i)]}")
-    return float((err / np.maximum(bound, 1e-30)).max())
+    ratio = float((err / np.maximum(bound, 1e-30)).max()) if err.size else 0.0
+    if ratio > WORST["ratio"]:
+        WORST["ratio"], WORST["what"] = ratio, what
+    return ratio
 
 
 @functools.lru_cache(maxsize=8)
