@@ -14,8 +14,11 @@
 //
 // One CTA computes 128 outputs for the whole batch over its share of K, in
 // 64-wide K steps:
-//   warp 0      TMA producer: x tiles (bf16, 128-byte swizzled, MT x 64) and
-//               packed code tiles (128 rows x 128 codes, unswizzled);
+//   warp 0      TMA producer of the packed code tiles (128 rows x 128 codes,
+//               unswizzled), as far ahead as the code ring allows;
+//   warp 10     TMA producer of the x tiles (bf16, 128-byte swizzled,
+//               MT x 64), which wait for the MMAs: kept apart so that the
+//               code stream (the HBM traffic) never waits on them;
 //   warp 1      owns tensor memory (MT fp32 columns x 128 lanes) and one lane
 //               issues the MMAs, A = W' from shared memory, B = x;
 //   warps 2..9  dequantise codes -> w' = bf16_rne(scale * (q - zero)) (exact
@@ -43,7 +46,8 @@ namespace {
 
 constexpr int BN = 128, BK = 64, CK = 128;
 constexpr int kDqWarps = 8;
-constexpr int kThreads = 64 + 32 * kDqWarps;
+constexpr int kXWarp = 2 + kDqWarps;                       // the x producer
+constexpr int kThreads = 32 * (kXWarp + 1);
 constexpr uint32_t kWBytes = uint32_t(BN) * BK * 2;       // one W' stage
 
 #ifndef WQ_GEMM_SW_MAX_SPLIT
@@ -53,19 +57,27 @@ constexpr uint32_t kWBytes = uint32_t(BN) * BK * 2;       // one W' stage
 #define WQ_GEMM_SW_MIN_STAGES 4   // 128-wide code stages each split keeps at least
 #endif
 
+// Scales and zeros reach the dequantising warps in chunks of kChG groups:
+// each warp copies its own 16 rows' windows (kChG halves plus an odd start,
+// kChW words per row and array) one chunk ahead into a double buffer.
+constexpr int kChG = 8;
+constexpr int kChW = kChG / 2 + 1;
+constexpr uint32_t kChWarpWords = 2u * 16 * 2 * kChW;              // [buffer][row][array][word]
+constexpr uint32_t kChBytes = kDqWarps * kChWarpWords * 4;
+
 template <int BITS, int MT>
 struct SwCfg {
   static constexpr uint32_t kXBytes = uint32_t(MT) * BK * 2;          // one x stage
   static constexpr uint32_t kCBytes = uint32_t(BN) * CK * BITS / 8;   // one code stage
-  static constexpr uint32_t kMisc = 1024 /* align */ + 512 /* barriers */ + 4 * BN /* row scales */;
-  // Two CTAs per SM when 3 W' stages, 2 x stages and 3 code stages fit in
+  static constexpr uint32_t kMisc = 1024 /* align */ + 512 /* barriers */ + 4 * BN /* row scales */ + kChBytes;
+  // Two CTAs per SM when 3 W' stages, 3 x stages and 3 code stages fit in
   // half the shared memory, else one CTA with deeper rings.  The code ring
   // (the HBM stream) takes what is left: the bandwidth an SM draws follows
   // the bytes it keeps in flight.
-  static constexpr bool kTwo = MT <= 128 && 3 * kWBytes + 2 * kXBytes + 3 * kCBytes + kMisc <= 112 * 1024;
+  static constexpr bool kTwo = MT <= 128 && 3 * kWBytes + 3 * kXBytes + 3 * kCBytes + kMisc <= 112 * 1024;
   static constexpr uint32_t kBudget = kTwo ? 112 * 1024 : 226 * 1024;
   static constexpr int SW = kTwo ? 3 : 4;
-  static constexpr int SX = kTwo ? 2 : (MT <= 128 ? 4 : 2);
+  static constexpr int SX = kTwo ? 3 : (MT <= 128 ? 4 : 2);
   static constexpr int SCf = int((kBudget - kMisc - SW * kWBytes - SX * kXBytes) / kCBytes);
   static constexpr int SC = SCf > 8 ? 8 : SCf;
   static_assert(SC >= 3, "code ring");
@@ -94,7 +106,8 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t* b, uint32_t bytes) {
                : "memory");
 }
 __device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, volatile uint32_t* abort) {
-  return bw::pipe_wait(smem_u32(b), parity, &g_gemm_sw_timeout, abort);
+  const uint32_t a = smem_u32(b);
+  return bw::try_parity(a, parity) || bw::pipe_wait(a, parity, &g_gemm_sw_timeout, abort);
 }
 __device__ __forceinline__ void mbar_drain(uint64_t* b, uint32_t parity) {
   bw::drain_wait(smem_u32(b), parity, &g_gemm_sw_timeout);
@@ -169,20 +182,34 @@ __device__ __forceinline__ uint32_t bf162_bits(float a, float b) {
   __nv_bfloat162 h = __floats2bfloat162_rn(a, b);   // a -> low half (lower address)
   return *reinterpret_cast<uint32_t*>(&h);
 }
-// bf16 pairs (codes 2j, 2j+1 of a unit) of w' = fma(q 2^-30, A, B), j = J..15:
-// the code from one AND is the subnormal q 2^(p-149); times 2^(119-p) it is
-// q 2^-30 exactly, and the FMA with A = s 2^30, B = -s z is exact (s q and
-// s z have at most 20 significant bits), so the bf16 conversion is the only
-// rounding.
+__device__ __forceinline__ uint64_t f32x2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+// bf16 pairs (codes 2j, 2j+1 of a unit) of w' = fma(q 2^-30, A, B), j = J..15,
+// two lanes of fp32 per packed multiply and FMA: the code from one AND is the
+// subnormal q 2^(p-149); times 2^(119-p) it is q 2^-30 exactly, and the FMA
+// with A = s 2^30, B = -s z is exact (s q and s z have at most 20 significant
+// bits), so the bf16 conversion is the only rounding.
 template <int BITS, int J>
 struct SwDq {
-  __device__ __forceinline__ static void run(const uint32_t (&w)[BITS], float A, float B, uint32_t (&out)[16]) {
+  __device__ __forceinline__ static void run(const uint32_t (&w)[BITS], uint64_t AA, uint64_t BB,
+                                             uint32_t (&out)[16]) {
     constexpr float F0 = pow2f(119 - code_p<BITS>(2 * J));
     constexpr float F1 = pow2f(119 - code_p<BITS>(2 * J + 1));
-    const float a = fmaf(code_subnormal<BITS, 2 * J>(w) * F0, A, B);
-    const float b = fmaf(code_subnormal<BITS, 2 * J + 1>(w) * F1, A, B);
-    out[J] = bf162_bits(a, b);
-    if constexpr (J + 1 < 16) SwDq<BITS, J + 1>::run(w, A, B, out);
+    const uint64_t q2 = f32x2(code_subnormal<BITS, 2 * J>(w), code_subnormal<BITS, 2 * J + 1>(w));
+    uint64_t v;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(v) : "l"(q2), "l"(f32x2(F0, F1)));
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(v) : "l"(v), "l"(AA), "l"(BB));
+    uint32_t o;
+    asm("{\n\t.reg .f32 lo, hi;\n\t"
+        "mov.b64 {lo, hi}, %1;\n\t"
+        "cvt.rn.bf16x2.f32 %0, hi, lo;\n\t}"
+        : "=r"(o)
+        : "l"(v));
+    out[J] = o;                                          // code 2j in the low half
+    if constexpr (J + 1 < 16) SwDq<BITS, J + 1>::run(w, AA, BB, out);
   }
 };
 template <int BITS>
@@ -204,7 +231,7 @@ __device__ __forceinline__ void lds_unit(const uint8_t* p, uint32_t (&w)[BITS]) 
   }
 }
 
-// Two resident CTAs of 10 warps put up to 6 warps on one of the SM's four
+// Two resident CTAs of 11 warps put up to 6 warps on one of the SM's four
 // schedulers, whose register file holds 16K registers: 80 per thread at most
 // (declared as a 384-thread bound for two CTAs).
 template <int BITS, int MT>
@@ -219,7 +246,8 @@ gemm_sw_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
   uint8_t* sX = base;                                   // [SX][MT x 64 bf16], swizzled
   uint8_t* sW = sX + SX * Cfg::kXBytes;                 // [SW][128 x 64 bf16], swizzled
   uint8_t* sC = sW + SW * kWBytes;                      // [SC][128 rows x 128 codes]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sC + SC * Cfg::kCBytes);
+  uint32_t* sCh = reinterpret_cast<uint32_t*>(sC + SC * Cfg::kCBytes);   // [kDqWarps][kChWarpWords]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sCh + kDqWarps * kChWarpWords);
   uint64_t* full_x = bars;             // TMA x landed             (1 arrival + bytes)
   uint64_t* empty_x = full_x + SX;     // MMAs done with the x slot (commit)
   uint64_t* full_w = empty_x + SX;     // W' written              (kDqWarps arrivals)
@@ -229,7 +257,7 @@ gemm_sw_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
   uint64_t* tmem_full = empty_c + SC;  // accumulators final       (commit)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tmem_full + 1);
   volatile uint32_t* abort = tmem_slot + 1;
-  float* row_scale = reinterpret_cast<float*>(base + Cfg::kRing + 512);   // [128], per-row grids
+  float* row_scale = reinterpret_cast<float*>(bars + 64);   // [128], per-row grids
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t n0 = int64_t(blockIdx.x) * BN;
@@ -269,31 +297,37 @@ gemm_sw_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
   bool ep_ok = false;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
+    // ------------------------------------------------------------ code producer
     if (lane == 0) {
-      int issued_x = 0, issued_c = 0;
+      const int nc = (kt1 - kt0 + 1) / 2;              // 128-wide code stages of this split
+      int issued = 0;
+      bool ok = true;
+      for (int c = 0; c < nc && ok; ++c) {
+        const int cs = c % SC;
+        if (c >= SC) ok = mbar_wait(&empty_c[cs], ((c / SC) - 1) & 1, abort);
+        if (!ok) break;
+        mbar_expect_tx(&full_c[cs], Cfg::kCBytes);
+        tma_load_2d(sC + cs * Cfg::kCBytes, &tm_c, &full_c[cs], ((kt0 >> 1) + c) * (CK * BITS / 32), int(n0));
+        ++issued;
+      }
+      if (!ok)   // copies in flight land before shared memory goes away
+        for (int c = (issued > SC ? issued - SC : 0); c < issued; ++c) mbar_drain(&full_c[c % SC], (c / SC) & 1);
+    }
+  } else if (warp == kXWarp) {
+    // ------------------------------------------------------------ x producer
+    if (lane == 0) {
+      int issued = 0;
       bool ok = true;
       for (int kt = kt0; kt < kt1 && ok; ++kt) {
-        const int j = kt - kt0;
-        if ((j & 1) == 0) {                              // codes for K [kt*64, kt*64 + 128)
-          const int c = j >> 1, cs = c % SC;
-          if (c >= SC) ok = mbar_wait(&empty_c[cs], ((c / SC) - 1) & 1, abort);
-          if (!ok) break;
-          mbar_expect_tx(&full_c[cs], Cfg::kCBytes);
-          tma_load_2d(sC + cs * Cfg::kCBytes, &tm_c, &full_c[cs], (kt >> 1) * (CK * BITS / 32), int(n0));
-          ++issued_c;
-        }
-        const int s = j % SX;
+        const int j = kt - kt0, s = j % SX;
         if (j >= SX) ok = mbar_wait(&empty_x[s], ((j / SX) - 1) & 1, abort);
         if (!ok) break;
         mbar_expect_tx(&full_x[s], Cfg::kXBytes);
         tma_load_2d(sX + s * Cfg::kXBytes, &tm_x, &full_x[s], kt * BK, 0);
-        ++issued_x;
+        ++issued;
       }
-      if (!ok) {   // copies in flight land before shared memory goes away
-        for (int j = (issued_x > SX ? issued_x - SX : 0); j < issued_x; ++j) mbar_drain(&full_x[j % SX], (j / SX) & 1);
-        for (int c = (issued_c > SC ? issued_c - SC : 0); c < issued_c; ++c) mbar_drain(&full_c[c % SC], (c / SC) & 1);
-      }
+      if (!ok)
+        for (int j = (issued > SX ? issued - SX : 0); j < issued; ++j) mbar_drain(&full_x[j % SX], (j / SX) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -316,7 +350,7 @@ gemm_sw_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
       }
       umma_commit(tmem_full);      // always: the teardown waits on it before freeing tensor memory
     }
-  } else {
+  } else if (warp < kXWarp) {
     // ------------------------------------------------------------ dequantise
     const int td = threadIdx.x - 64;                 // 0..255
     const int r = td >> 1, cu = td & 1;              // tile row, 32-code unit of the 64-wide step
@@ -326,39 +360,76 @@ gemm_sw_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
       if (cu == 0) row_scale[r] = n < N ? __half2float(scales[n * G]) : 0.0f;
       asm volatile("bar.sync 1, %0;" ::"n"(32 * kDqWarps) : "memory");
     }
-    const unsigned short* srow = n < N ? reinterpret_cast<const unsigned short*>(scales) + n * G : nullptr;
-    const unsigned short* zrow = (n < N && zeros) ? reinterpret_cast<const unsigned short*>(zeros) + n * G : nullptr;
-    // scale and zero of step kt as raw fp16 bits (the symmetric grid's zero when no array)
-    auto load_raw = [&](int kt, uint16_t& s2, uint16_t& z2) {
-      const int k = kt * BK + 32 * cu;
-      const uint32_t grp = units_per_group.div(uint32_t(k < K ? k >> 5 : 0));
-      s2 = 0;
-      z2 = 0;
-      if (kt < kt1 && srow != nullptr && k < K) {
-        s2 = rowwise ? uint16_t(0x3C00) : __ldg(srow + grp);      // 0x3C00: fp16 1.0
-        z2 = zrow ? __ldg(zrow + grp) : uint16_t((BITS - 1 + 15) << 10);
+    // per-row grids: the zero of the row, once (the scale goes to the epilogue)
+    const uint16_t zsym = uint16_t((BITS - 1 + 15) << 10);   // fp16 2^(b-1): the symmetric grid's zero
+    uint16_t rz2 = zsym;
+    if (rowwise && zeros && n < N) rz2 = __ldg(reinterpret_cast<const unsigned short*>(zeros) + n * G);
+    // grouped grids: chunk q holds groups [grp0 + 8 q, grp0 + 8 q + 8) of the
+    // warp's rows; lane l copies array l & 1 (scales, zeros) of row l / 2
+    const int dw = warp - 2;
+    uint32_t* chw = sCh + dw * kChWarpWords;
+    const uint32_t grp0 = rowwise ? 0u : units_per_group.div(uint32_t((kt0 * BK) >> 5));
+    const uint32_t gend = rowwise ? 0u : units_per_group.div(uint32_t((kt1 * BK - 1) >> 5)) + 1u;
+    auto load_chunk = [&](int qc) {
+      const int rr = 16 * dw + (lane >> 1), arr = lane & 1;
+      const int64_t nn = n0 + rr;
+      const __half* src = arr ? zeros : scales;
+      const uint32_t ga = grp0 + uint32_t(qc) * kChG;
+      const uint32_t gb = min(ga + uint32_t(kChG), gend);
+      if (src != nullptr && nn < N && ga < gb) {
+        const int64_t e0 = nn * G + ga, a0 = e0 & ~int64_t(1), end = N * G;
+        const int nw = int((e0 + (gb - ga) - a0 + 1) >> 1);
+        const uint32_t dst = smem_u32(chw + (((qc & 1) * 16 + (lane >> 1)) * 2 + arr) * kChW);
+        for (int w = 0; w < nw; ++w) {
+          const int64_t a = a0 + 2 * w;                  // a < end: the window ends at a needed group
+          const uint32_t bytes = a + 2 <= end ? 4u : 2u;
+          asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst + 4 * w), "l"(src + a), "r"(bytes)
+                       : "memory");
+        }
       }
+      asm volatile("cp.async.commit_group;" ::: "memory");
     };
+    if (!rowwise) load_chunk(0);
+    int qcur = -1;
     bool ok = true;
-    uint16_t cs2, cz2, ns2 = 0, nz2 = 0;
-    load_raw(kt0, cs2, cz2);
     for (int kt = kt0; kt < kt1 && ok; ++kt) {
-      load_raw(kt + 1, ns2, nz2);                    // next step's, one step ahead
-      const float sc = __half2float(__ushort_as_half(cs2));
-      const float A = sc * 0x1p30f, B = -sc * __half2float(__ushort_as_half(cz2));
       const int j = kt - kt0;
       const int c = j >> 1, cs = c % SC, s = j % SW;
       ok = mbar_wait(&full_c[cs], (c / SC) & 1, abort);
       if (ok && j >= SW) ok = mbar_wait(&empty_w[s], ((j / SW) - 1) & 1, abort);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
+      // scale and zero of this thread's 32 codes as raw fp16 bits: element h
+      // of the row's window in the chunk (h = the parity of the window's first
+      // element + the group's offset in the chunk)
+      uint16_t s2 = 0x3C00, z2 = rz2;                   // 0x3C00: fp16 1.0
+      if (!rowwise) {
+        const int q = int((units_per_group.div(uint32_t((kt * BK) >> 5)) - grp0) / kChG);   // warp-uniform
+        if (q != qcur) {
+          __syncwarp();                                  // every lane is done with chunk q - 1's buffer
+          if (grp0 + uint32_t(q + 1) * kChG < gend) load_chunk(q + 1);
+          else asm volatile("cp.async.commit_group;" ::: "memory");
+          asm volatile("cp.async.wait_group 1;" ::: "memory");   // chunk q has landed (this lane's part)
+          __syncwarp();                                  // ... and every lane's
+          qcur = q;
+        }
+        const uint32_t ga = grp0 + uint32_t(q) * kChG;
+        const uint32_t h = uint32_t((n * G + ga) & 1) + units_per_group.div(uint32_t((kt * BK + 32 * cu) >> 5)) - ga;
+        const unsigned short* ch =
+            reinterpret_cast<const unsigned short*>(chw + (((q & 1) * 16 + (lane >> 1)) * 2) * kChW);
+        s2 = ch[h];
+        z2 = zeros ? ch[2 * kChW + h] : zsym;
+      }
+      const float sc = __half2float(__ushort_as_half(s2));
+      const float A = sc * 0x1p30f, B = -sc * __half2float(__ushort_as_half(z2));
+      const uint64_t AA = f32x2(A, A), BB = f32x2(B, B);
       const uint8_t* ctile = sC + cs * Cfg::kCBytes;
       uint8_t* wtile = sW + s * kWBytes;
       const int ucode = (kt & 1) * 2 + cu;           // unit within the 128-code stage
       uint32_t w[BITS];
       lds_unit<BITS>(ctile + r * (CK * BITS / 8) + ucode * (4 * BITS), w);
       uint32_t p[16];
-      SwDq<BITS, 0>::run(w, A, B, p);
+      SwDq<BITS, 0>::run(w, AA, BB, p);
       uint8_t* wrow = wtile + r * 128;
 #pragma unroll
       for (int jj = 0; jj < 4; ++jj) {
@@ -371,65 +442,87 @@ gemm_sw_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         mbar_arrive(&full_w[s]);
         if ((j & 1) || kt == kt1 - 1) mbar_arrive(&empty_c[cs]);
       }
-      cs2 = ns2;
-      cz2 = nz2;
     }
+    asm volatile("cp.async.wait_all;" ::: "memory");   // no copy may land after the CTA exits
     if (ok) ok = mbar_wait(tmem_full, 0, abort);
     ep_ok = __all_sync(0xffffffffu, ok);             // tcgen05.ld needs the whole warp
   }
 
   // ------------------------------------------------------------ epilogue
   // Warp w (2..9) reads tensor-memory lane quarter w % 4 (rows 32 (w % 4) ..)
-  // and column half (w - 2) / 4.  With split-K, ranks > 0 first park their
-  // partial tile in their own (now idle) shared memory as [column / 4][row][4]
-  // floats and rank 0 adds them through distributed shared memory.  Every
-  // thread takes part in the cluster barriers.
-  const bool dq = warp >= 2;
+  // and column half (w - 2) / 4.  Without split-K it converts its columns to
+  // bf16 and stores them.  With split-K every rank parks its fp32 partial tile
+  // in its own (now idle) shared memory as [column / 4][row][4] floats; then
+  // rank r sums the 4-column groups u = r, r + ks, ... over all ranks (in
+  // rank order, through distributed shared memory) and stores them, so the
+  // reduction is spread over the cluster.  Every thread takes part in the
+  // cluster barriers.
+  const bool dq = warp >= 2 && warp < kXWarp;
   const int q = warp & 3, ch = (warp - 2) >> 2;
   const int row = 32 * q + lane;
   const int64_t n = n0 + row;
   float4* part = reinterpret_cast<float4*>(sX);
   const uint32_t tbase = tmem + (uint32_t(32 * q) << 16);
   constexpr int HALF = MT / 2;
-  if (ks > 1 && kr != 0 && dq && ep_ok) {
-    tc_fence_after();
+  if (ks == 1) {
+    if (dq && ep_ok) {
+      tc_fence_after();
+      const float rs = rowwise ? row_scale[row] : 1.0f;
 #pragma unroll 1
-    for (int c0 = ch * HALF; c0 < (ch + 1) * HALF; c0 += 16) {
-      float v[16];
-      tmem_ld16(tbase + uint32_t(c0), v);
+      for (int c0 = ch * HALF; c0 < (ch + 1) * HALF; c0 += 16) {
+        float v[16];
+        tmem_ld16(tbase + uint32_t(c0), v);
+        if (n < N) {
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
-        part[((c0 >> 2) + u) * BN + row] = make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
-    }
-  }
-  if (ks > 1) cluster_sync();
-  if (kr == 0 && dq && ep_ok) {
-    tc_fence_after();
-    const float rs = rowwise ? row_scale[row] : 1.0f;
-#pragma unroll 1
-    for (int c0 = ch * HALF; c0 < (ch + 1) * HALF; c0 += 16) {
-      float v[16];
-      tmem_ld16(tbase + uint32_t(c0), v);
-      for (int pr = 1; pr < ks; ++pr) {
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float4 pv = ld_peer_f4(&part[((c0 >> 2) + u) * BN + row], pr);
-          v[4 * u] += pv.x;
-          v[4 * u + 1] += pv.y;
-          v[4 * u + 2] += pv.z;
-          v[4 * u + 3] += pv.w;
-        }
-      }
-      if (n < N) {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int64_t m = c0 + i;
-          if (m < M) y[m * N + n] = __float2bfloat16_rn(rowwise ? v[i] * rs : v[i]);
+          for (int i = 0; i < 16; ++i) {
+            const int64_t m = c0 + i;
+            if (m < M) y[m * N + n] = __float2bfloat16_rn(rowwise ? v[i] * rs : v[i]);
+          }
         }
       }
     }
+  } else {
+    if (dq && ep_ok) {
+      tc_fence_after();
+#pragma unroll 1
+      for (int c0 = ch * HALF; c0 < (ch + 1) * HALF; c0 += 16) {
+        float v[16];
+        tmem_ld16(tbase + uint32_t(c0), v);
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          part[((c0 >> 2) + u) * BN + row] = make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+      }
+    }
+    cluster_sync();
+    if (dq) {
+      const float rs = rowwise ? row_scale[row] : 1.0f;
+#pragma unroll 1
+      for (int u = kr + ks * ch; u < MT / 4; u += 2 * ks) {
+        float4 pv[WQ_GEMM_SW_MAX_SPLIT];
+#pragma unroll
+        for (int pr = 0; pr < WQ_GEMM_SW_MAX_SPLIT; ++pr)
+          if (pr < ks) pv[pr] = ld_peer_f4(&part[u * BN + row], pr);   // all loads in flight at once
+        float4 v = pv[0];
+#pragma unroll
+        for (int pr = 1; pr < WQ_GEMM_SW_MAX_SPLIT; ++pr)
+          if (pr < ks) {
+            v.x += pv[pr].x;
+            v.y += pv[pr].y;
+            v.z += pv[pr].z;
+            v.w += pv[pr].w;
+          }
+        if (n < N) {
+          const float o[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int64_t m = 4 * u + i;
+            if (m < M) y[m * N + n] = __float2bfloat16_rn(rowwise ? o[i] * rs : o[i]);
+          }
+        }
+      }
+    }
+    cluster_sync();                                  // peers keep their partials until read
   }
-  if (ks > 1) cluster_sync();                        // peers keep their partials until read
 
   // ------------------------------------------------------------ teardown
   tc_fence_before();
@@ -445,25 +538,12 @@ gemm_sw_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
 }
 
 // ------------------------------------------------------------------ host
-constexpr double kWaveStages = 4.0;    // prologue + epilogue of one wave, in code stages
-constexpr double kSplitStages = 1.5;   // partial-tile exchange per extra split
-
-// Resident CTAs of this configuration per SM (cached per device).
-template <int BITS, int MT>
-int blocks_per_sm(int dev) {
-  static std::atomic<int> cache[64];
-  if (dev < 0 || dev >= 64) return 1;
-  int v = cache[dev].load(std::memory_order_relaxed);
-  if (v == 0) {
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, gemm_sw_kernel<BITS, MT>, kThreads,
-                                                      SwCfg<BITS, MT>::kSmem) != cudaSuccess || v < 1) {
-      cudaGetLastError();
-      v = 1;
-    }
-    cache[dev].store(v, std::memory_order_relaxed);
-  }
-  return v;
-}
+#ifndef WQ_GEMM_SW_SPLIT_STAGES
+#define WQ_GEMM_SW_SPLIT_STAGES 1.0
+#endif
+constexpr double kWaveStages = 4.0;    // prologue + epilogue of one CTA, in code stages
+constexpr double kSplitStages = WQ_GEMM_SW_SPLIT_STAGES;   // partial-tile exchange per extra split
+constexpr double kPairGain = 1.35;     // throughput of an SM running two CTAs, relative to one
 
 template <int BITS, int MT>
 cudaError_t launch_mt(const __nv_bfloat16* x, int64_t M, int64_t N, int64_t K, const uint32_t* codes,
@@ -481,23 +561,35 @@ cudaError_t launch_mt(const __nv_bfloat16* x, int64_t M, int64_t N, int64_t K, c
   if (!attr_set[dev].load(std::memory_order_acquire)) {
     cudaError_t e = cudaFuncSetAttribute(gemm_sw_kernel<BITS, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          int(Cfg::kSmem));
+    // all of the unified L1 as shared memory: the two-CTA builds need it
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(gemm_sw_kernel<BITS, MT>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                               int(cudaSharedmemCarveoutMaxShared));
     if (e != cudaSuccess) return e;
     attr_set[dev].store(true, std::memory_order_release);
   }
-  // Split K over a cluster when the 128-row tiles alone fill the SMs badly
-  // (cost in units of one 128-wide code stage, cluster slots per wave from
-  // the occupancy API).
+  // Split K over a cluster when the 128-row tiles alone fill the SMs badly.
+  // Cost in units of one 128-wide code stage: a CTA takes its share of K
+  // plus a fixed prologue/epilogue and an exchange cost per extra split; an
+  // SM that holds two CTAs (the two-CTA builds) runs each at kPairGain / 2
+  // of the speed of one.  The resident CTAs per SM come from the build (the
+  // runtime's occupancy query reports one CTA per SM for the two-CTA
+  // builds, which ncu and the launches show resident in pairs).
   const int64_t tiles = (N + BN - 1) / BN;
   const int64_t kc = K / CK;
   int nsm = 0;
   if (cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || nsm < 1) nsm = 1;
-  const int64_t slots = int64_t(nsm) * blocks_per_sm<BITS, MT>(dev);   // CTA slots per wave
   int ks = 1;
   double best = 1e300;
   for (int c = 1; c <= WQ_GEMM_SW_MAX_SPLIT; ++c) {
     if (c > 1 && kc / c < WQ_GEMM_SW_MIN_STAGES) break;
-    const double waves = double((tiles * c + slots - 1) / slots);
-    const double t = waves * (double(kc) / c + kWaveStages + kSplitStages * (c - 1));
+    const int64_t n = tiles * c;
+    const double per_cta = double(kc) / c + kWaveStages + kSplitStages * (c - 1);
+    double t;
+    if (Cfg::kTwo && n > nsm)
+      t = double((n + 2 * nsm - 1) / (2 * nsm)) * 2.0 * per_cta / kPairGain;
+    else
+      t = double((n + nsm - 1) / nsm) * per_cta;
     if (t < best - 1e-9) {
       best = t;
       ks = c;

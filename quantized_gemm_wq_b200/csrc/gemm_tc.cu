@@ -181,17 +181,33 @@ constexpr float pow2f(int e) {
 
 __device__ __forceinline__ uint32_t bf162_bits(float a, float b);
 
-// bf16 pairs (codes 2j, 2j+1 of a unit) of w' = fma(q 2^-30, A, B), j = J..15.
+__device__ __forceinline__ uint64_t f32x2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+
+// bf16 pairs (codes 2j, 2j+1 of a unit) of w' = fma(q 2^-30, A, B), j = J..15,
+// two codes per packed fp32 multiply and FMA (the same IEEE operations as
+// two scalar ones); AA, BB hold A and B in both lanes.
 template <int BITS, int J>
 struct DqPairs {
-  __device__ __forceinline__ static void run(const uint32_t (&w)[BITS], float A, float B,
+  __device__ __forceinline__ static void run(const uint32_t (&w)[BITS], uint64_t AA, uint64_t BB,
                                              uint32_t (&out)[16]) {
     constexpr float F0 = pow2f(119 - code_p<BITS>(2 * J));
     constexpr float F1 = pow2f(119 - code_p<BITS>(2 * J + 1));
-    const float a = fmaf(code_subnormal<BITS, 2 * J>(w) * F0, A, B);
-    const float b = fmaf(code_subnormal<BITS, 2 * J + 1>(w) * F1, A, B);
-    out[J] = bf162_bits(a, b);
-    if constexpr (J + 1 < 16) DqPairs<BITS, J + 1>::run(w, A, B, out);
+    const uint64_t q2 = f32x2(code_subnormal<BITS, 2 * J>(w), code_subnormal<BITS, 2 * J + 1>(w));
+    uint64_t v;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(v) : "l"(q2), "l"(f32x2(F0, F1)));
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(v) : "l"(v), "l"(AA), "l"(BB));
+    uint32_t o;
+    asm("{\n\t.reg .f32 lo, hi;\n\t"
+        "mov.b64 {lo, hi}, %1;\n\t"
+        "cvt.rn.bf16x2.f32 %0, hi, lo;\n\t}"
+        : "=r"(o)
+        : "l"(v));
+    out[J] = o;                                          // code 2j in the low half
+    if constexpr (J + 1 < 16) DqPairs<BITS, J + 1>::run(w, AA, BB, out);
   }
 };
 
@@ -416,7 +432,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         uint32_t w[BITS];
         lds_unit<BITS>(ctile + r * (CK * BITS / 8) + ucode * (4 * BITS), w);
         uint32_t p[16];
-        DqPairs<BITS, 0>::run(w, A[i], B[i], p);
+        DqPairs<BITS, 0>::run(w, f32x2(A[i], A[i]), f32x2(B[i], B[i]), p);
         uint8_t* brow = btile + r * 128;
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) {
