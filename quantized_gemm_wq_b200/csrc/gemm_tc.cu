@@ -468,20 +468,61 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
 
   // ------------------------------------------------------------ epilogue
   // Accumulator mt (rows 128 mt .. 128 mt + 127 of the tile) is written out by
-  // the 8 dequant warps: warp w reads TMEM lane quarter w % 4 and 128 of the 256
-  // columns.  With split-K, ranks > 0 first park their partial tile in their
-  // own (now idle) shared memory as [column / 4][row][4] floats, and rank 0
-  // adds them in through distributed shared memory.  Every thread takes part
-  // in the cluster barriers.
+  // the 8 dequant warps: warp w reads TMEM lane quarter w % 4.  Without
+  // split-K, warp w converts 128 of the 256 columns and stores them.  With
+  // split-K every rank parks its partial tile in its own (now idle) shared
+  // memory as [column / 4][row][4] floats; then rank r sums the 32-column
+  // blocks b = r, r + ks, ... over all ranks (in rank order, through
+  // distributed shared memory) and stores them, so the reduction is spread
+  // over the cluster.  Every thread takes part in the cluster barriers.
   const bool dq = warp >= 2;
   const int q = warp & 3;                    // TMEM lane quarter this warp may access
-  const int ch = (warp - 2) >> 2;            // column half
+  const int ch = (warp - 2) >> 2;            // column half / block parity
   float4* part = reinterpret_cast<float4*>(sA);
   const bool vec = (N % 8) == 0;
+  // bf16 of 32 columns of row m from column n, scaled per column for per-row grids
+  auto store32 = [&](int64_t m, int col0, uint32_t (&r)[32]) {
+    if (rowwise) {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) * col_scale[col0 + j]);
+    }
+    const int64_t n = n0 + col0;
+    if (m < M && n < N) {
+      __nv_bfloat16* dst = y + m * N + n;
+      if (vec && n + 32 <= N) {
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          uint4 o;
+          o.x = bf162_bits(__uint_as_float(r[8 * v + 0]), __uint_as_float(r[8 * v + 1]));
+          o.y = bf162_bits(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3]));
+          o.z = bf162_bits(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5]));
+          o.w = bf162_bits(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7]));
+          reinterpret_cast<uint4*>(dst)[v] = o;
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (n + j < N) dst[j] = __float2bfloat16_rn(__uint_as_float(r[j]));
+      }
+    }
+  };
   for (int mt = 0; mt < BM / kMmaM; ++mt) {
     const int row = 32 * q + lane;           // row within accumulator mt
+    const int64_t m = m0 + mt * kMmaM + row;
     const uint32_t tbase = tmem + (uint32_t(32 * q) << 16) + uint32_t(mt * kMmaN);
-    if (ks > 1 && kr != 0 && dq && ep_ok) {
+    if (ks == 1) {
+      if (dq && ep_ok) {
+        tc_fence_after();
+        for (int cb = 0; cb < 4; ++cb) {
+          const int col0 = 128 * ch + 32 * cb;
+          uint32_t r[32];
+          tmem_ld32(tbase + uint32_t(col0), r);
+          store32(m, col0, r);
+        }
+      }
+      continue;
+    }
+    if (dq && ep_ok) {
       tc_fence_after();
       for (int cb = 0; cb < 4; ++cb) {
         const int col0 = 128 * ch + 32 * cb;
@@ -494,51 +535,37 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                           __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
       }
     }
-    if (ks > 1) cluster_sync();
-    if (kr == 0 && dq && ep_ok) {
-      tc_fence_after();
-      const int64_t m = m0 + mt * kMmaM + row;
-      for (int cb = 0; cb < 4; ++cb) {
-        const int col0 = 128 * ch + 32 * cb;
-        uint32_t r[32];
-        tmem_ld32(tbase + uint32_t(col0), r);
+    cluster_sync();
+    if (dq) {
+      for (int blk = kr + ks * ch; blk < kMmaN / 32; blk += 2 * ks) {
+        const int col0 = 32 * blk;
+        float4 acc[8];
+#pragma unroll
+        for (int v = 0; v < 8; ++v) acc[v] = ld_peer_f4(&part[((col0 >> 2) + v) * 128 + row], 0);
         for (int pr = 1; pr < ks; ++pr) {
+          float4 pv[8];
+#pragma unroll
+          for (int v = 0; v < 8; ++v) pv[v] = ld_peer_f4(&part[((col0 >> 2) + v) * 128 + row], pr);
 #pragma unroll
           for (int v = 0; v < 8; ++v) {
-            const float4 pv = ld_peer_f4(&part[((col0 >> 2) + v) * 128 + row], pr);
-            r[4 * v] = __float_as_uint(__uint_as_float(r[4 * v]) + pv.x);
-            r[4 * v + 1] = __float_as_uint(__uint_as_float(r[4 * v + 1]) + pv.y);
-            r[4 * v + 2] = __float_as_uint(__uint_as_float(r[4 * v + 2]) + pv.z);
-            r[4 * v + 3] = __float_as_uint(__uint_as_float(r[4 * v + 3]) + pv.w);
+            acc[v].x += pv[v].x;
+            acc[v].y += pv[v].y;
+            acc[v].z += pv[v].z;
+            acc[v].w += pv[v].w;
           }
         }
-        if (rowwise) {
+        uint32_t r[32];
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
-            r[j] = __float_as_uint(__uint_as_float(r[j]) * col_scale[col0 + j]);
+        for (int v = 0; v < 8; ++v) {
+          r[4 * v] = __float_as_uint(acc[v].x);
+          r[4 * v + 1] = __float_as_uint(acc[v].y);
+          r[4 * v + 2] = __float_as_uint(acc[v].z);
+          r[4 * v + 3] = __float_as_uint(acc[v].w);
         }
-        const int64_t n = n0 + col0;
-        if (m < M && n < N) {
-          __nv_bfloat16* dst = y + m * N + n;
-          if (vec && n + 32 <= N) {
-#pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              uint4 o;
-              o.x = bf162_bits(__uint_as_float(r[8 * v + 0]), __uint_as_float(r[8 * v + 1]));
-              o.y = bf162_bits(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3]));
-              o.z = bf162_bits(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5]));
-              o.w = bf162_bits(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7]));
-              reinterpret_cast<uint4*>(dst)[v] = o;
-            }
-          } else {
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (n + j < N) dst[j] = __float2bfloat16_rn(__uint_as_float(r[j]));
-          }
-        }
+        store32(m, col0, r);
       }
     }
-    if (ks > 1) cluster_sync();              // peers keep their partials until read
+    cluster_sync();                          // peers keep their partials until read
   }
 
   // ------------------------------------------------------------ teardown
@@ -556,16 +583,18 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
 
 // ------------------------------------------------------------------ host
 constexpr double kWaveStages = 5.0;    // prologue + epilogue of one wave, in code stages
-constexpr double kSplitStages = 3.0;   // partial-tile exchange per extra split
+#ifndef WQ_GEMM_SPLIT_STAGES
+#define WQ_GEMM_SPLIT_STAGES 1.5
+#endif
+constexpr double kSplitStages = WQ_GEMM_SPLIT_STAGES;   // partial-tile exchange per extra split
 
 // Clusters of c CTAs (one per SM, `smem` bytes each) resident at once; cached
 // per device and cluster size.  0 if the query fails.
 template <int BITS>
 int cluster_slots(int dev, int c, uint32_t smem) {
-  static std::atomic<int> cache[64][4];   // 0 unknown, -1 query failed
-  int ci = 0;
-  while ((1 << ci) < c) ++ci;
-  if (dev < 0 || dev >= 64 || ci > 3) return 0;
+  static std::atomic<int> cache[64][WQ_GEMM_MAX_SPLIT + 1];   // 0 unknown, -1 query failed
+  const int ci = c;
+  if (dev < 0 || dev >= 64 || ci < 1 || ci > WQ_GEMM_MAX_SPLIT) return 0;
   const int known = cache[dev][ci].load(std::memory_order_relaxed);
   if (known != 0) return known > 0 ? known : 0;
   cudaLaunchConfig_t cfg = {};
@@ -619,7 +648,7 @@ cudaError_t launch_bits(const __nv_bfloat16* x, int64_t M, int64_t N, int64_t K,
   const int64_t kc = K / CK;
   int ks = 1;
   double best = 1e300;
-  for (int c = 1; c <= WQ_GEMM_MAX_SPLIT; c *= 2) {
+  for (int c = 1; c <= WQ_GEMM_MAX_SPLIT; ++c) {
     if (c > 1 && kc / c < WQ_GEMM_MIN_STAGES) break;
     const int slots = cluster_slots<BITS>(dev, c, smem);
     if (slots <= 0) break;
