@@ -51,7 +51,12 @@ constexpr int BM = 256, BN = 256, BK = 64, CK = 128;
 #define WQ_GEMM_MIN_STAGES 8  // 128-wide code stages each split keeps at least
 #endif
 constexpr int kMmaM = 128, kMmaN = 256, kMmaK = 16;
-constexpr int kDqWarps = 8;
+#ifndef WQ_GEMM_DQ_WARPS
+#define WQ_GEMM_DQ_WARPS 8
+#endif
+constexpr int kDqWarps = WQ_GEMM_DQ_WARPS;                 // 8 or 16
+constexpr int kRowsPerThread = BN / (16 * kDqWarps);       // W' rows each dequantising thread writes
+constexpr int kColGroups = kDqWarps / 4;                   // epilogue column groups per TMEM lane quarter
 constexpr int kThreads = 64 + 32 * kDqWarps;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kABytes = BM * BK * 2;
@@ -91,7 +96,8 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t* b, uint32_t bytes) {
 // Waits: bounded_wait.cuh (pipeline waits give up after its limit, raising
 // the CTA abort word and g_timeout_flag; exit-path drains ignore the abort).
 __device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, volatile uint32_t* abort) {
-  return bw::pipe_wait(smem_u32(b), parity, &g_timeout_flag, abort);
+  const uint32_t a = smem_u32(b);
+  return bw::try_parity(a, parity) || bw::pipe_wait(a, parity, &g_timeout_flag, abort);
 }
 __device__ __forceinline__ void mbar_drain(uint64_t* b, uint32_t parity) {
   bw::drain_wait(smem_u32(b), parity, &g_timeout_flag);
@@ -364,11 +370,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
     const int64_t G = K / g;
     if (rowwise) {                           // epilogue scale of each output column
       const int c = threadIdx.x - 64;
-      col_scale[c] = (n0 + c < N) ? __half2float(scales[(n0 + c) * G]) : 0.0f;
+      if (c < BN) col_scale[c] = (n0 + c < N) ? __half2float(scales[(n0 + c) * G]) : 0.0f;
       asm volatile("bar.sync 1, %0;" ::"n"(32 * kDqWarps) : "memory");
     }
-    // Per thread: rows r0 = 32 dw + lane / 2 and r0 + 16 of the tile, unit cu of
-    // every 64-wide K step.  w' = s (q - z) = fma(q 2^-30, s 2^30, -s z): the
+    // Per thread: rows 16 (dw + kDqWarps i) + lane / 2 of the tile
+    // (i < kRowsPerThread), unit cu of every 64-wide K step.  w' = s (q - z) = fma(q 2^-30, s 2^30, -s z): the
     // code comes out of one AND as the subnormal float q 2^(p-149), one FMUL by
     // 2^(119-p) (exact) gives q 2^-30, and the FMA is exact (s q and s z have at
     // most 20 significant bits); the bf16 conversion is the only rounding.
@@ -376,21 +382,21 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
     // bits; nothing reads those registers until that step (a use right after
     // the load would stall the warp for the whole load latency), so the loop
     // runs two steps per iteration with two register sets.
-    const int r0 = 32 * dw + (lane >> 1);
+    const int r0 = 16 * dw + (lane >> 1);
     // This thread's two rows of the scale and zero arrays (row n >= N: none).
-    const unsigned short* srow[2];
-    const unsigned short* zrow[2];
+    const unsigned short* srow[kRowsPerThread];
+    const unsigned short* zrow[kRowsPerThread];
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const int64_t n = n0 + r0 + 16 * i;
+    for (int i = 0; i < kRowsPerThread; ++i) {
+      const int64_t n = n0 + r0 + 16 * kDqWarps * i;
       srow[i] = n < N ? reinterpret_cast<const unsigned short*>(scales) + n * G : nullptr;
       zrow[i] = n < N && zeros ? reinterpret_cast<const unsigned short*>(zeros) + n * G : nullptr;
     }
-    auto load_raw = [&](int kt, uint16_t (&s2)[2], uint16_t (&z2)[2]) {
+    auto load_raw = [&](int kt, uint16_t (&s2)[kRowsPerThread], uint16_t (&z2)[kRowsPerThread]) {
       const int k = kt * BK + 32 * cu;
       const uint32_t grp = units_per_group.div(uint32_t(k < K ? k >> 5 : 0));
 #pragma unroll
-      for (int i = 0; i < 2; ++i) {
+      for (int i = 0; i < kRowsPerThread; ++i) {
         s2[i] = 0;
         z2[i] = 0;
         if (kt < kt1 && srow[i] != nullptr && k < K) {
@@ -407,12 +413,12 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
     bool ok = true;
     // One K step with the step's raw scale/zero (cs, cz); the next step's are
     // requested into (ns, nz).
-    auto step = [&](int kt, const uint16_t (&cs2)[2], const uint16_t (&cz2)[2], uint16_t (&ns2)[2],
-                    uint16_t (&nz2)[2], bool load_next) {
+    auto step = [&](int kt, const uint16_t (&cs2)[kRowsPerThread], const uint16_t (&cz2)[kRowsPerThread],
+                    uint16_t (&ns2)[kRowsPerThread], uint16_t (&nz2)[kRowsPerThread], bool load_next) {
       if (load_next) load_raw(kt + 1, ns2, nz2);
-      float A[2], B[2];
+      float A[kRowsPerThread], B[kRowsPerThread];
 #pragma unroll
-      for (int i = 0; i < 2; ++i) {
+      for (int i = 0; i < kRowsPerThread; ++i) {
         const float sc = __half2float(__ushort_as_half(cs2[i]));
         A[i] = sc * 0x1p30f;
         B[i] = -sc * __half2float(__ushort_as_half(cz2[i]));
@@ -427,8 +433,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
       uint8_t* btile = sB + s * kBBytes;
       const int ucode = (kt & 1) * 2 + cu;   // unit index within the 128-code stage
 #pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        const int r = r0 + 16 * i;
+      for (int i = 0; i < kRowsPerThread; ++i) {
+        const int r = r0 + 16 * kDqWarps * i;
         uint32_t w[BITS];
         lds_unit<BITS>(ctile + r * (CK * BITS / 8) + ucode * (4 * BITS), w);
         uint32_t p[16];
@@ -447,7 +453,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         if ((j & 1) || kt == kt1 - 1) mbar_arrive(&empty_c[cs]);
       }
     };
-    uint16_t s0r[2], z0r[2], s1r[2], z1r[2];
+    uint16_t s0r[kRowsPerThread], z0r[kRowsPerThread], s1r[kRowsPerThread], z1r[kRowsPerThread];
     load_raw(kt0, s0r, z0r);
     if (pair_group) {
       for (int kt = kt0; kt < kt1 && ok; kt += 4) {   // two pairs: register sets 0 then 1
@@ -477,7 +483,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
   // over the cluster.  Every thread takes part in the cluster barriers.
   const bool dq = warp >= 2;
   const int q = warp & 3;                    // TMEM lane quarter this warp may access
-  const int ch = (warp - 2) >> 2;            // column half / block parity
+  const int ch = (warp - 2) >> 2;            // column group (kColGroups of them)
   float4* part = reinterpret_cast<float4*>(sA);
   const bool vec = (N % 8) == 0;
   // bf16 of 32 columns of row m from column n, scaled per column for per-row grids
@@ -513,8 +519,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
     if (ks == 1) {
       if (dq && ep_ok) {
         tc_fence_after();
-        for (int cb = 0; cb < 4; ++cb) {
-          const int col0 = 128 * ch + 32 * cb;
+        for (int cb = 0; cb < 8 / kColGroups; ++cb) {
+          const int col0 = (256 / kColGroups) * ch + 32 * cb;
           uint32_t r[32];
           tmem_ld32(tbase + uint32_t(col0), r);
           store32(m, col0, r);
@@ -524,8 +530,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
     }
     if (dq && ep_ok) {
       tc_fence_after();
-      for (int cb = 0; cb < 4; ++cb) {
-        const int col0 = 128 * ch + 32 * cb;
+      for (int cb = 0; cb < 8 / kColGroups; ++cb) {
+        const int col0 = (256 / kColGroups) * ch + 32 * cb;
         uint32_t r[32];
         tmem_ld32(tbase + uint32_t(col0), r);
 #pragma unroll
@@ -537,7 +543,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
     }
     cluster_sync();
     if (dq) {
-      for (int blk = kr + ks * ch; blk < kMmaN / 32; blk += 2 * ks) {
+      for (int blk = kr + ks * ch; blk < kMmaN / 32; blk += kColGroups * ks) {
         const int col0 = 32 * blk;
         float4 acc[8];
 #pragma unroll

@@ -24,4 +24,6 @@ def pytest_terminal_summary(terminalreporter):
     mod = sys.modules.get("gpu_util")
     if mod is not None and mod.WORST["ratio"] > 0.0:
         terminalreporter.write_line(
-            f"parity: max |y - y_ref| / sum|x w'| = {mod.WORST['ratio']:.3e} ({mod.WORST['what']})")
+            f"parity: max |y - y_ref| / sum|x w'| = {mod.WORST['ratio']:.3e} ({mod.WORST['what']}); "
+            f"largest share of the tolerance 2e-3 sum|x w'| + 2^-8 |y| + 1e-3 used = "
+            f"{mod.WORST['used']:.3f} ({mod.WORST['used_what']})")

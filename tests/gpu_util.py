@@ -42,8 +42,9 @@ def oracle_quantize(Wh: np.ndarray, bits: int, group: int):
 
 
 # Largest max |y - y_ref| / sum_k |x w'| seen by assert_y_close in this run,
-# with the check that produced it (printed in the pytest summary).
-WORST = {"ratio": 0.0, "what": ""}
+# and the largest share of the per-element tolerance used, each with the check
+# that produced it (printed in the pytest summary).
+WORST = {"ratio": 0.0, "what": "", "used": 0.0, "used_what": ""}
 
 
 def assert_y_close(y_gpu: np.ndarray, y_ref: np.ndarray, bound: np.ndarray, what: str = ""):
@@ -56,8 +57,11 @@ def assert_y_close(y_gpu: np.ndarray, y_ref: np.ndarray, bound: np.ndarray, what
                              f"{tuple(i)} gpu={y_gpu[tuple(i)]} ref={y_ref[tuple(i)]} "
                              f"bound={bound[tuple(i)]}")
     ratio = float((err / np.maximum(bound, 1e-30)).max()) if err.size else 0.0
+    used = float((err / lim).max()) if err.size else 0.0
     if ratio > WORST["ratio"]:
         WORST["ratio"], WORST["what"] = ratio, what
+    if used > WORST["used"]:
+        WORST["used"], WORST["used_what"] = used, what
     return ratio
 
 
