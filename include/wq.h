@@ -202,10 +202,13 @@ typedef struct {
  * that never drains between tiles or linears.  A short preparation kernel
  * first writes each x, pre-scaled for the tensor cores, into the workspace.
  * The multiply-adds run on warp-level MMAs (mma.sync, bf16 in, fp32 out),
- * with the same exact products and the same accuracy bound as wq_gemm.  Other
- * linears (and every linear when M > 16) run as wq_gemm would run them.
- * Every argument of every linear is checked before anything is launched, as
- * for wq_gemm; outputs must not overlap any input or each other.
+ * with the same exact products and the same accuracy bound as wq_gemm.
+ * For 17 <= M <= 255, linears whose K is a multiple of 128 run the swap-AB
+ * tensor-core GEMM of wq_gemm in one launch per 64 linears, one CTA per
+ * 128-row tile over all of K (no workspace is needed).  Other linears run as
+ * wq_gemm would run them.  Every argument of every linear is checked before
+ * anything is launched, as for wq_gemm; outputs must not overlap any input or
+ * each other.
  */
 wq_status wq_gemm_grouped(const wq_linear* linears, int count, int64_t M, int bits, void* workspace,
                           size_t workspace_bytes, void* stream);

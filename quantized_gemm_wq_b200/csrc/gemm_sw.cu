@@ -36,6 +36,7 @@
 #include <atomic>
 
 #include "bounded_wait.cuh"
+#include "grouped.h"
 #include "wq_internal.cuh"
 
 namespace wq {
@@ -60,6 +61,7 @@ constexpr uint32_t kWBytes = uint32_t(BN) * BK * 2;       // one W' stage
 // Scales and zeros reach the dequantising warps in chunks of kChG groups:
 // each warp copies its own 16 rows' windows (kChG halves plus an odd start,
 // kChW words per row and array) one chunk ahead into a double buffer.
+constexpr int kMaxSwLinears = 64;   // linears per grouped launch (kernel parameter space)
 constexpr int kChG = 8;
 constexpr int kChW = kChG / 2 + 1;
 constexpr uint32_t kChWarpWords = 2u * 16 * 2 * kChW;              // [buffer][row][array][word]
@@ -90,6 +92,22 @@ struct SwCfg {
       (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(MT >> 3) << 17) | (uint32_t(BN >> 4) << 24);
   static_assert(kPartBytes <= kRing, "the partial tile is parked in the ring");
   static_assert(kSmem <= 227 * 1024, "shared memory");
+};
+
+// One linear of a grouped launch (tensor maps first: they need 64-byte alignment).
+struct alignas(64) SwLin {
+  CUtensorMap tm_x, tm_c;
+  const __half* scales;
+  const __half* zeros;
+  __nv_bfloat16* y;
+  int64_t N, K, g;
+  FastDiv upg;
+  int tile0;        // first CTA of this linear's row tiles
+};
+struct SwGroup {
+  SwLin lin[kMaxSwLinears];
+  int nlin;
+  int64_t M;
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -231,14 +249,13 @@ __device__ __forceinline__ void lds_unit(const uint8_t* p, uint32_t (&w)[BITS]) 
   }
 }
 
-// Two resident CTAs of 11 warps put up to 6 warps on one of the SM's four
-// schedulers, whose register file holds 16K registers: 80 per thread at most
-// (declared as a 384-thread bound for two CTAs).
+// One CTA's work: output rows n0 .. n0 + 127 of one linear over split kr of
+// ks along K (the tensor maps live in kernel parameter space).
 template <int BITS, int MT>
-__global__ void __launch_bounds__(SwCfg<BITS, MT>::kTwo ? 384 : kThreads, SwCfg<BITS, MT>::kTwo ? 2 : 1)
-gemm_sw_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_c,
-               const __half* __restrict__ scales, const __half* __restrict__ zeros, int64_t M, int64_t N,
-               int64_t K, int64_t g, FastDiv units_per_group, __nv_bfloat16* __restrict__ y) {
+__device__ __forceinline__ void sw_tile(const CUtensorMap* tm_x, const CUtensorMap* tm_c,
+                                        const __half* __restrict__ scales, const __half* __restrict__ zeros,
+                                        int64_t M, int64_t N, int64_t K, int64_t g, FastDiv units_per_group,
+                                        __nv_bfloat16* __restrict__ y, int64_t n0, int ks, int kr) {
   using Cfg = SwCfg<BITS, MT>;
   constexpr int SX = Cfg::SX, SW = Cfg::SW, SC = Cfg::SC;
   extern __shared__ uint8_t smem_raw[];
@@ -260,9 +277,7 @@ gemm_sw_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
   float* row_scale = reinterpret_cast<float*>(bars + 64);   // [128], per-row grids
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t n0 = int64_t(blockIdx.x) * BN;
   const int KT = int((K + BK - 1) / BK);
-  const int ks = int(gridDim.z), kr = int(blockIdx.z);
   const int KC = (KT + 1) / 2;
   const int kt0 = 2 * int(int64_t(KC) * kr / ks);
   const int kt1 = min(KT, 2 * int(int64_t(KC) * (kr + 1) / ks));
@@ -307,7 +322,7 @@ gemm_sw_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         if (c >= SC) ok = mbar_wait(&empty_c[cs], ((c / SC) - 1) & 1, abort);
         if (!ok) break;
         mbar_expect_tx(&full_c[cs], Cfg::kCBytes);
-        tma_load_2d(sC + cs * Cfg::kCBytes, &tm_c, &full_c[cs], ((kt0 >> 1) + c) * (CK * BITS / 32), int(n0));
+        tma_load_2d(sC + cs * Cfg::kCBytes, tm_c, &full_c[cs], ((kt0 >> 1) + c) * (CK * BITS / 32), int(n0));
         ++issued;
       }
       if (!ok)   // copies in flight land before shared memory goes away
@@ -323,7 +338,7 @@ gemm_sw_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         if (j >= SX) ok = mbar_wait(&empty_x[s], ((j / SX) - 1) & 1, abort);
         if (!ok) break;
         mbar_expect_tx(&full_x[s], Cfg::kXBytes);
-        tma_load_2d(sX + s * Cfg::kXBytes, &tm_x, &full_x[s], kt * BK, 0);
+        tma_load_2d(sX + s * Cfg::kXBytes, tm_x, &full_x[s], kt * BK, 0);
         ++issued;
       }
       if (!ok)
@@ -537,6 +552,36 @@ gemm_sw_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
   }
 }
 
+// Two resident CTAs of 11 warps put up to 6 warps on one of the SM's four
+// schedulers, whose register file holds 16K registers: 80 per thread at most
+// (declared as a 384-thread bound for two CTAs).
+#define WQ_SW_BOUNDS __launch_bounds__(SwCfg<BITS, MT>::kTwo ? 384 : kThreads, SwCfg<BITS, MT>::kTwo ? 2 : 1)
+
+// One linear: blockIdx.x the 128-row tile, blockIdx.z the split of K (a
+// cluster of gridDim.z CTAs along K).
+template <int BITS, int MT>
+__global__ void WQ_SW_BOUNDS gemm_sw_kernel(const __grid_constant__ CUtensorMap tm_x,
+                                            const __grid_constant__ CUtensorMap tm_c,
+                                            const __half* __restrict__ scales, const __half* __restrict__ zeros,
+                                            int64_t M, int64_t N, int64_t K, int64_t g, FastDiv units_per_group,
+                                            __nv_bfloat16* __restrict__ y) {
+  sw_tile<BITS, MT>(&tm_x, &tm_c, scales, zeros, M, N, K, g, units_per_group, y, int64_t(blockIdx.x) * BN,
+                    int(gridDim.z), int(blockIdx.z));
+}
+
+// Many linears in one launch: CTA b takes row tile b - tile0 of the linear
+// whose tiles hold b, over the whole of K (with thousands of tiles in a
+// decode step the SMs stay busy without splitting K).
+template <int BITS, int MT>
+__global__ void WQ_SW_BOUNDS gemm_sw_grouped_kernel(const __grid_constant__ SwGroup p) {
+  const int b = int(blockIdx.x);
+  int l = 0;
+  while (l + 1 < p.nlin && p.lin[l + 1].tile0 <= b) ++l;
+  const SwLin& L = p.lin[l];
+  sw_tile<BITS, MT>(&L.tm_x, &L.tm_c, L.scales, L.zeros, p.M, L.N, L.K, L.g, L.upg, L.y,
+                    int64_t(b - L.tile0) * BN, 1, 0);
+}
+
 // ------------------------------------------------------------------ host
 #ifndef WQ_GEMM_SW_SPLIT_STAGES
 #define WQ_GEMM_SW_SPLIT_STAGES 1.0
@@ -620,9 +665,73 @@ cudaError_t launch_bits(const __nv_bfloat16* x, int64_t M, int64_t N, int64_t K,
   return launch_mt<BITS, 256>(x, M, N, K, codes, scales, zeros, g, y, st);
 }
 
+template <int BITS, int MT>
+cudaError_t launch_grouped_mt(const GroupedLinear* lins, int count, int64_t M, cudaStream_t st) {
+  using Cfg = SwCfg<BITS, MT>;
+  static std::atomic<bool> attr_set[64];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!attr_set[dev].load(std::memory_order_acquire)) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_sw_grouped_kernel<BITS, MT>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, int(Cfg::kSmem));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(gemm_sw_grouped_kernel<BITS, MT>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                               int(cudaSharedmemCarveoutMaxShared));
+    if (e != cudaSuccess) return e;
+    attr_set[dev].store(true, std::memory_order_release);
+  }
+  SwGroup p;
+  for (int c0 = 0; c0 < count; c0 += kMaxSwLinears) {
+    const int n = count - c0 < kMaxSwLinears ? count - c0 : kMaxSwLinears;
+    p.nlin = n;
+    p.M = M;
+    int tiles = 0;
+    for (int j = 0; j < n; ++j) {
+      const GroupedLinear& L = lins[c0 + j];
+      SwLin& d = p.lin[j];
+      if (!make_tensor_map_2d(&d.tm_x, TmaType::kBF16, L.x, uint64_t(L.K), uint64_t(M), uint64_t(L.K) * 2, BK, MT,
+                              128) ||
+          !make_tensor_map_2d(&d.tm_c, TmaType::kU32, L.codes, uint64_t(L.K * BITS / 32), uint64_t(L.N),
+                              uint64_t(L.K * BITS / 8), CK * BITS / 32, BN, 0))
+        return cudaErrorInvalidValue;
+      d.scales = L.scales;
+      d.zeros = L.zeros;
+      d.y = L.y;
+      d.N = L.N;
+      d.K = L.K;
+      d.g = L.group;
+      d.upg = FastDiv(uint32_t(L.group / 32));
+      d.tile0 = tiles;
+      tiles += int((L.N + BN - 1) / BN);
+    }
+    gemm_sw_grouped_kernel<BITS, MT><<<dim3(unsigned(tiles)), dim3(kThreads), Cfg::kSmem, st>>>(p);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+template <int BITS>
+cudaError_t launch_grouped_bits(const GroupedLinear* lins, int count, int64_t M, cudaStream_t st) {
+  if (M <= 32) return launch_grouped_mt<BITS, 32>(lins, count, M, st);
+  if (M <= 64) return launch_grouped_mt<BITS, 64>(lins, count, M, st);
+  if (M <= 128) return launch_grouped_mt<BITS, 128>(lins, count, M, st);
+  return launch_grouped_mt<BITS, 256>(lins, count, M, st);
+}
+
 }  // namespace
 
 bool gemm_sw_supported(int64_t M, int64_t K) { return M > 16 && M < 256 && K % CK == 0; }
+
+cudaError_t launch_gemm_sw_grouped(const GroupedLinear* lins, int count, int64_t M, int bits, cudaStream_t st) {
+  switch (bits) {
+    case 2: return launch_grouped_bits<2>(lins, count, M, st);
+    case 3: return launch_grouped_bits<3>(lins, count, M, st);
+    case 4: return launch_grouped_bits<4>(lins, count, M, st);
+    default: return launch_grouped_bits<8>(lins, count, M, st);
+  }
+}
 
 cudaError_t launch_gemm_sw(const __nv_bfloat16* x, int64_t M, int64_t N, int64_t K, const uint32_t* codes,
                            const __half* scales, const __half* zeros, int bits, int64_t g, __nv_bfloat16* y,

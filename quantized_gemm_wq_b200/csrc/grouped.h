@@ -81,6 +81,11 @@ cudaError_t launch_gemv_grouped(const GroupedLinear* lins, int count, int M, int
                                 cudaStream_t st);
 bool gemv_grouped_read_and_clear_timeout(cudaError_t* err);
 
+// 17 <= M <= 255 (gemm_sw_supported): the swap-AB tensor-core GEMM over many
+// linears in one launch per 64 linears, one CTA per 128-row tile over all of K
+// (gemm_sw.cu).  No workspace.
+cudaError_t launch_gemm_sw_grouped(const GroupedLinear* lins, int count, int64_t M, int bits, cudaStream_t st);
+
 // The built-in workspace of wq_gemm_grouped_noalloc (noalloc.cu): its size,
 // and its device address on the current device (looked up on first use).
 size_t static_workspace_bytes();

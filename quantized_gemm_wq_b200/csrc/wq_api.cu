@@ -94,6 +94,23 @@ wq::GroupedLinear to_grouped(const wq_linear& L) {
                            static_cast<__nv_bfloat16*>(L.y_bf16), L.N, L.K, wq::effective_group(L.K, L.group)};
 }
 
+// The linears of a grouped call that the swap-AB GEMM takes in grouped
+// launches (17 <= M <= 255, K a multiple of 128).
+std::vector<wq::GroupedLinear> grouped_sw_list(const wq_linear* lins, int count, int64_t M) {
+  std::vector<wq::GroupedLinear> v;
+  if (M <= wq::kGemvMaxM) return v;
+  for (int i = 0; i < count; ++i) {
+    const wq::GroupedLinear g = to_grouped(lins[i]);
+    if (wq::gemm_sw_supported(M, g.K)) v.push_back(g);
+  }
+  return v;
+}
+
+// True when linear L of a grouped call runs in one of the grouped launches.
+bool grouped_launch_takes(const wq::GroupedLinear& g, int64_t M) {
+  return M <= wq::kGemvMaxM ? wq::grouped_supported(g.K, g.group) : wq::gemm_sw_supported(M, g.K);
+}
+
 // The linears of a grouped call that the persistent kernel takes.
 std::vector<wq::GroupedLinear> grouped_fast_list(const wq_linear* lins, int count, int64_t M) {
   std::vector<wq::GroupedLinear> v;
@@ -217,9 +234,11 @@ wq_status wq_gemm_grouped(const wq_linear* linears, int count, int64_t M, int bi
   const auto strm = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaSuccess;
   if (!fast.empty()) e = wq::launch_gemv_grouped(fast.data(), int(fast.size()), int(M), bits, ws, strm);
+  const std::vector<wq::GroupedLinear> sw = grouped_sw_list(linears, count, M);
+  if (e == cudaSuccess && !sw.empty()) e = wq::launch_gemm_sw_grouped(sw.data(), int(sw.size()), M, bits, strm);
   for (int i = 0; i < count && e == cudaSuccess; ++i) {
     const wq::GroupedLinear g = to_grouped(linears[i]);
-    if (M <= wq::kGemvMaxM && wq::grouped_supported(g.K, g.group)) continue;
+    if (grouped_launch_takes(g, M)) continue;
     e = dispatch_one(g.x, M, g.N, g.K, g.codes, g.scales, g.zeros, bits, g.group, g.y, strm);
   }
   return e == cudaSuccess ? WQ_OK : WQ_ERR_CUDA;
@@ -252,9 +271,11 @@ wq_status wq_gemm_grouped_noalloc(const wq_linear* linears, int count, int64_t M
     e = cudaMemsetAsync(ws.cnt, 0, sizeof(unsigned) * wq::kMaxCtas, strm);
     if (e == cudaSuccess) e = wq::launch_gemv_grouped(fast.data(), int(fast.size()), int(M), bits, ws, strm);
   }
+  const std::vector<wq::GroupedLinear> sw = grouped_sw_list(linears, count, M);
+  if (e == cudaSuccess && !sw.empty()) e = wq::launch_gemm_sw_grouped(sw.data(), int(sw.size()), M, bits, strm);
   for (int i = 0; i < count && e == cudaSuccess; ++i) {
     const wq::GroupedLinear g = to_grouped(linears[i]);
-    if (M <= wq::kGemvMaxM && wq::grouped_supported(g.K, g.group)) continue;
+    if (grouped_launch_takes(g, M)) continue;
     e = dispatch_one(g.x, M, g.N, g.K, g.codes, g.scales, g.zeros, bits, g.group, g.y, strm);
   }
   return e == cudaSuccess ? WQ_OK : WQ_ERR_CUDA;

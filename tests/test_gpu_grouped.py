@@ -1,7 +1,8 @@
-"""Grouped decode GEMV (wq_gemm_grouped) vs the oracle: every y of a list of
-linears within the stated tolerance, one-hot exactness, determinism, stream-K
-splits of a tile between CTAs, several launches sharing one workspace, and
-nothing written outside y."""
+"""Grouped calls (wq_gemm_grouped) vs the oracle: every y of a list of linears
+within the stated tolerance, one-hot exactness, determinism, stream-K splits of
+a tile between CTAs, several launches sharing one workspace, nothing written
+outside y; at 1..16 rows the persistent decode GEMV, at 17..255 rows the
+swap-AB tensor-core GEMM in grouped launches."""
 from __future__ import annotations
 
 import numpy as np
@@ -177,3 +178,65 @@ def test_grouped_no_write_outside_y_and_small_workspace_refused():
     torch.cuda.synchronize()
     assert torch.all(buf[:32] == 7.0) and torch.all(buf[32 + 2 * N:] == 7.0)
     _check_all([(Wh, c, s, z, N, K, group)], [x.cpu()], [y], bits, "canaries")
+
+
+# 17..255 rows: the swap-AB tensor-core GEMM in grouped launches (one CTA per
+# 128-row tile over all of K); the K = 96 linear still runs as wq_gemm would.
+@pytest.mark.parametrize("bits", BITS)
+@pytest.mark.parametrize("M", [17, 33, 64, 100, 255])
+def test_grouped_swap_ab(bits, M):
+    qs = _quantized(26, SHAPES, bits, dist="t4")
+    xs = [wq_inputs.activations_bf16(26, 500 + i, M, K) for i, (_, K, _) in enumerate(SHAPES)]
+    m = wq()
+    items = [(x.cuda(), c, s, z, N, K, g) for x, (_, c, s, z, N, K, g) in zip(xs, qs)]
+    ys = m.wq_gemm_grouped(items, bits)
+    torch.cuda.synchronize()
+    _check_all(qs, xs, ys, bits, f"swap-AB grouped bits={bits} M={M}")
+
+
+@pytest.mark.parametrize("bits", (2, 4, 8))
+def test_grouped_swap_ab_one_hot_exact(bits):
+    """One-hot tokens (the last all zero) through the grouped swap-AB launch:
+    y must equal bf16(c w') exactly, per-row and grouped grids."""
+    shapes = [(200, 1152, 128), (130, 2048, 0)]
+    qs = _quantized(27, shapes, bits)
+    M = 40
+    m = wq()
+    items, refs = [], []
+    for (Wh, c, s, z, N, K, group) in qs:
+        oc, os_, oz = oracle_quantize(Wh, bits, group)
+        w_ref = oracle.dequant(oracle.unpack(oc, K, bits), os_, oz, group)
+        x = torch.zeros(M, K, dtype=torch.bfloat16)
+        r = []
+        for i in range(M - 1):
+            k = (37 * i + 5) % K
+            v = 2.0 if i % 2 else -1.0
+            x[i, k] = v
+            r.append((i, (v * torch.from_numpy(w_ref[:, k])).to(torch.bfloat16)))
+        refs.append(r)
+        items.append((x.cuda(), c, s, z, N, K, group))
+    ys = [y.cpu() for y in m.wq_gemm_grouped(items, bits)]
+    for y, r in zip(ys, refs):
+        for i, want in r:
+            assert torch.equal(y[i], want), f"token {i}"
+        assert torch.all(y[M - 1] == 0)
+
+
+def test_grouped_swap_ab_many_linears_and_noalloc():
+    """150 linears at 48 rows: three grouped launches (at most 64 linears
+    each); the no-alloc entry gives the same bits (no workspace is used)."""
+    bits = 4
+    shapes = [(64 + (i % 7) * 40, 128 * (1 + i % 6), 128 if i % 4 else 0) for i in range(150)]
+    qs = _quantized(28, shapes, bits)
+    m = wq()
+    M = 48
+    xs = [wq_inputs.activations_bf16(28, 600 + i, M, K) for i, (_, K, _) in enumerate(shapes)]
+    items = [(x.cuda(), c, s, z, N, K, g) for x, (_, c, s, z, N, K, g) in zip(xs, qs)]
+    ys = m.wq_gemm_grouped(items, bits)
+    torch.cuda.synchronize()
+    _check_all(qs, xs, ys, bits, "150 linears at 48 rows")
+    items2 = [it + (torch.empty(M, it[4], dtype=torch.bfloat16, device="cuda"),) for it in items]
+    ys2 = m.wq_gemm_grouped_noalloc(items2, bits)
+    torch.cuda.synchronize()
+    for a, b in zip(ys, ys2):
+        assert torch.equal(a, b)
