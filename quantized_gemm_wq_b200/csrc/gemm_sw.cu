@@ -73,13 +73,15 @@ struct SwCfg {
   static constexpr uint32_t kCBytes = uint32_t(BN) * CK * BITS / 8;   // one code stage
   static constexpr uint32_t kMisc = 1024 /* align */ + 512 /* barriers */ + 4 * BN /* row scales */ + kChBytes;
   // Two CTAs per SM when 3 W' stages, 3 x stages and 3 code stages fit in
-  // half the shared memory, else one CTA with deeper rings.  The code ring
-  // (the HBM stream) takes what is left: the bandwidth an SM draws follows
-  // the bytes it keeps in flight.
-  static constexpr bool kTwo = MT <= 128 && 3 * kWBytes + 3 * kXBytes + 3 * kCBytes + kMisc <= 112 * 1024;
+  // half the shared memory, or else 2, 2 and 3; otherwise one CTA with
+  // deeper rings.  The code ring (the HBM stream) takes what is left: the
+  // bandwidth an SM draws follows the bytes it keeps in flight.
+  static constexpr bool kTwo3 = MT <= 128 && 3 * kWBytes + 3 * kXBytes + 3 * kCBytes + kMisc <= 112 * 1024;
+  static constexpr bool kTwo2 = MT <= 128 && 2 * kWBytes + 2 * kXBytes + 3 * kCBytes + kMisc <= 112 * 1024;
+  static constexpr bool kTwo = kTwo3 || kTwo2;
   static constexpr uint32_t kBudget = kTwo ? 112 * 1024 : 226 * 1024;
-  static constexpr int SW = kTwo ? 3 : 4;
-  static constexpr int SX = kTwo ? 3 : (MT <= 128 ? 4 : 2);
+  static constexpr int SW = kTwo3 ? 3 : (kTwo2 ? 2 : 4);
+  static constexpr int SX = kTwo3 ? 3 : (kTwo2 ? 2 : (MT <= 128 ? 4 : 2));
   static constexpr int SCf = int((kBudget - kMisc - SW * kWBytes - SX * kXBytes) / kCBytes);
   static constexpr int SC = SCf > 8 ? 8 : SCf;
   static_assert(SC >= 3, "code ring");
