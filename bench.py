@@ -598,7 +598,7 @@ def main(argv=None):
                     help="measure the headline leg only (the stack at M = 1, 4, 16, 64)")
     ap.add_argument("--case", default=None,
                     help="run one small profiling case instead of the benchmark: "
-                         "stack:<M>:<layers> | gemv:<i> | gemv16:<i> | prefill:<i>")
+                         "stack:<M>:<layers> | stackpl:<M>:<layers> | gemv:<i> | gemv16:<i> | prefill:<i>")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -620,14 +620,15 @@ def main(argv=None):
 def run_case(case: str) -> None:
     """One small profiling case (for ncu), after 3 untimed repetitions:
     ``stack:<M>:<layers>`` one decode step over the first <layers> layers of
-    the 32-layer stack (layers >= 2 exceed L2): one wq_gemm_grouped call for
-    M <= 16, one wq_gemm per linear above; ``gemv:<i>`` /
+    the 32-layer stack (layers >= 2 exceed L2) as one wq_gemm_grouped call
+    (``stackpl:`` the same as one wq_gemm per linear); ``gemv:<i>`` /
     ``gemv16:<i>`` one wq_gemm of projection i of the 3-bit layer at M = 1 / 16;
     ``prefill:<i>`` one prefill GEMM (M = 2048) of the 13B-shaped workload."""
     import torch
     import quantized_gemm_wq_b200 as wq
     kind, _, arg = case.partition(":")
-    if kind == "stack":
+    if kind in ("stack", "stackpl"):
+        per_linear = kind == "stackpl"
         Ms, _, nl = arg.partition(":")
         M, layers = int(Ms or 1), int(nl or 4)
         w = wq_inputs.WORKLOADS[HEADLINE]
@@ -637,13 +638,13 @@ def run_case(case: str) -> None:
             c, s, z = wq.wq_quantize_rtn(W, w["bits"], w["group"])
             del W
             items.append((device_x(0, li, M, K), c, s, z, N, K, w["group"]))
-        ws = wq.grouped_workspace(items, w["bits"]) if M <= 16 else None
+        ws = wq.grouped_workspace(items, w["bits"])
         for _ in range(4):
-            if M <= 16:
-                wq.wq_gemm_grouped(items, w["bits"], workspace=ws)
-            else:
+            if per_linear:
                 for (x, c, s, z, N, K, g) in items:
                     wq.wq_gemm(x, c, s, z, w["bits"], g, N, K)
+            else:
+                wq.wq_gemm_grouped(items, w["bits"], workspace=ws)
         torch.cuda.synchronize()
         assert wq.wq_last_device_error() == wq.WQ_OK
         print(json.dumps({"case": case, "linears": len(items), "ok": True}))

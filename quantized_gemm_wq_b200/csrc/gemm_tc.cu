@@ -246,7 +246,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_c,
                const __half* __restrict__ scales, const __half* __restrict__ zeros, int64_t M,
                int64_t N, int64_t K, int64_t g, FastDiv units_per_group,
-               __nv_bfloat16* __restrict__ y) {
+               __nv_bfloat16* __restrict__ y, int tile0, int ntn) {
   using Cfg = TcCfg<BITS>;
   constexpr int SX = Cfg::kXStages, SW = Cfg::kWStages, SC = Cfg::kCStages;
   extern __shared__ uint8_t smem_raw[];
@@ -268,7 +268,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
   float* col_scale = reinterpret_cast<float*>(tmem_slot + 2);   // [BN], per-row grids only
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t n0 = int64_t(blockIdx.x) * BN, m0 = int64_t(blockIdx.y) * BM;
+  // output tile t = tile0 + blockIdx.x, row-major over (M tiles, N tiles)
+  const int t = tile0 + int(blockIdx.x);
+  const int64_t n0 = int64_t(t % ntn) * BN, m0 = int64_t(t / ntn) * BM;
   const int KT = int((K + BK - 1) / BK);
   // Split-K over the CTAs of a cluster (gridDim.z of them): this CTA takes the
   // 128-wide code stages [cb, ce), i.e. K steps [kt0, kt1); the partial tiles
@@ -650,35 +652,66 @@ cudaError_t launch_bits(const __nv_bfloat16* x, int64_t M, int64_t N, int64_t K,
   // takes its share of K plus a fixed prologue/epilogue and a reduction cost
   // per extra split; the cluster slots per wave come from the occupancy API
   // (clusters of c CTAs of this size do not always pack the SMs fully).
-  const int64_t tiles = ((N + BN - 1) / BN) * ((M + BM - 1) / BM);
+  // Besides one launch for all tiles, the model weighs two: the whole waves
+  // of tiles without a split, then the few tiles left over split over
+  // clusters (so that a last, nearly empty wave of whole tiles does not set
+  // the time).
+  const int ntn = int((N + BN - 1) / BN);
+  const int tiles = ntn * int((M + BM - 1) / BM);
   const int64_t kc = K / CK;
-  int ks = 1;
-  double best = 1e300;
-  for (int c = 1; c <= WQ_GEMM_MAX_SPLIT; ++c) {
-    if (c > 1 && kc / c < WQ_GEMM_MIN_STAGES) break;
+  auto cost = [&](int ntiles, int c) -> double {
     const int slots = cluster_slots<BITS>(dev, c, smem);
-    if (slots <= 0) break;
-    const double waves = double((tiles + slots - 1) / slots);
-    const double t = waves * (double(kc) / c + kWaveStages + kSplitStages * (c - 1));
-    if (t < best - 1e-9) {
-      best = t;
-      ks = c;
+    if (slots <= 0) return 1e300;
+    const double waves = double((ntiles + slots - 1) / slots);
+    return waves * (double(kc) / c + kWaveStages + kSplitStages * (c - 1));
+  };
+  auto best_split = [&](int ntiles, double* t_out) -> int {
+    int bc = 1;
+    double bt = 1e300;
+    for (int c = 1; c <= WQ_GEMM_MAX_SPLIT; ++c) {
+      if (c > 1 && kc / c < WQ_GEMM_MIN_STAGES) break;
+      const double t = cost(ntiles, c);
+      if (t < bt - 1e-9) {
+        bt = t;
+        bc = c;
+      }
+    }
+    *t_out = bt;
+    return bc;
+  };
+  double t_one = 0.0;
+  const int ks_one = best_split(tiles, &t_one);
+  const int slots1 = cluster_slots<BITS>(dev, 1, smem);
+  int whole = 0, ks_rest = 1;
+  if (slots1 > 0 && tiles > slots1 && tiles % slots1 != 0) {
+    const int w = (tiles / slots1) * slots1;
+    double t_rest = 0.0;
+    const int c = best_split(tiles - w, &t_rest);
+    if (double(w / slots1) * (double(kc) + kWaveStages) + t_rest < t_one - 1e-9) {
+      whole = w;
+      ks_rest = c;
     }
   }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(unsigned((N + BN - 1) / BN), unsigned((M + BM - 1) / BM), unsigned(ks));
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 1;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = unsigned(ks);
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BITS>, tx, tc, scales, zeros, M, N, K, g,
-                            FastDiv(uint32_t(g / 32)), y);
+  auto launch = [&](int tile0, int count, int ks) -> cudaError_t {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(unsigned(count), 1, unsigned(ks));
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = unsigned(ks);
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BITS>, tx, tc, scales, zeros, M, N, K, g,
+                              FastDiv(uint32_t(g / 32)), y, tile0, ntn);
+  };
+  if (whole == 0) return launch(0, tiles, ks_one);
+  cudaError_t e = launch(0, whole, 1);
+  if (e == cudaSuccess) e = launch(whole, tiles - whole, ks_rest);
+  return e;
 }
 
 }  // namespace

@@ -85,3 +85,23 @@ def test_tc_full_size_sampled(cfg, linear, M):
     xs = x[torch.from_numpy(rows)]
     y_ref, bound = oracle.gemm(wq_inputs.bf16_bits(xs), oc, os_, oz, len(cols), K, bits, group)
     assert_y_close(y[np.ix_(rows, cols)], y_ref, bound, f"{cfg}/{name} M={M}")
+
+
+@pytest.mark.parametrize("bits,group", [(4, 128), (3, 0)])
+def test_tc_whole_waves_then_split_rest(bits, group):
+    """152 tiles of 256 x 256 on 148 SMs: one launch of 148 whole tiles, then
+    the 4 left over with K split over a cluster.  Rows of the first and the
+    last row of tiles, columns of every tile, against the oracle."""
+    M, N, K = 2048, 4864, 2048
+    Wh = wq_inputs.weight_f16(31, 0, N, K)
+    x = wq_inputs.activations_bf16(31, 1, M, K)
+    m = wq()
+    codes, s, z = m.wq_quantize_rtn(to_dev_f16(Wh), bits, group)
+    y = m.wq_gemm(x.cuda(), codes, s, z, bits, group, N, K).float().cpu().numpy()
+    assert m.wq_last_device_error() == m.WQ_OK
+    rng = np.random.default_rng(10)
+    cols = np.unique(np.concatenate([np.arange(0, N, 256), np.arange(255, N, 256), rng.integers(0, N, 40)]))
+    rows = np.unique(np.concatenate([[0, 255, 1792, M - 1], rng.integers(0, 256, 6), rng.integers(1792, M, 10)]))
+    oc, os_, oz = oracle_quantize(Wh[cols], bits, group)
+    y_ref, bound = oracle.gemm(wq_inputs.bf16_bits(x[torch.from_numpy(rows)]), oc, os_, oz, len(cols), K, bits, group)
+    assert_y_close(y[np.ix_(rows, cols)], y_ref, bound, f"152 tiles bits={bits} g={group}")
