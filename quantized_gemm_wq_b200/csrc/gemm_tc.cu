@@ -45,7 +45,7 @@ namespace {
 constexpr int BM = 256, BN = 256, BK = 64, CK = 128;
 
 #ifndef WQ_GEMM_MAX_SPLIT
-#define WQ_GEMM_MAX_SPLIT 4   // largest split-K cluster
+#define WQ_GEMM_MAX_SPLIT 8   // largest split-K cluster
 #endif
 #ifndef WQ_GEMM_MIN_STAGES
 #define WQ_GEMM_MIN_STAGES 8  // 128-wide code stages each split keeps at least
