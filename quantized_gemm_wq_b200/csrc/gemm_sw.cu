@@ -26,11 +26,13 @@
 //               swizzled layout, then the epilogue: tcgen05.ld -> bf16 -> y.
 // With one grid per row the MMA gets the exact integers q - zero and the fp32
 // scale of each row (tensor-memory lane) is applied in the epilogue.
-// K is split over a thread-block cluster when the 128-row tiles leave SMs
-// idle; ranks > 0 park their fp32 partial tile in their own shared memory and
-// rank 0 adds them through distributed shared memory.  Every wait is bounded
-// (bounded_wait.cuh): an expired wait raises this file's device flag, the CTA
-// drains its copies and MMAs and frees its tensor memory.
+// One linear (gemm_sw_kernel): K is split over a thread-block cluster when
+// the 128-row tiles leave SMs idle; every rank parks its fp32 partial tile in
+// its own shared memory and each rank sums a share of the columns over all
+// ranks through distributed shared memory.  Many linears
+// (gemm_sw_grouped_kernel): one launch over all their row tiles, K not split.
+// Every wait is bounded (bounded_wait.cuh): an expired wait raises this file's
+// device flag, the CTA drains its copies and MMAs and frees its tensor memory.
 #include <cuda.h>
 
 #include <atomic>
