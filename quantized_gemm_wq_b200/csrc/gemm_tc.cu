@@ -7,7 +7,11 @@
 // contraction, so it runs on the tensor cores with W' rebuilt in bf16 on chip.
 //
 // One CTA computes a 256 x 256 tile of y (256 batch rows x 256 output
-// features) over the whole K, in 64-wide K steps:
+// features) over its share of K, in 64-wide K steps (the whole K, or a share
+// of it when K is split over a thread-block cluster: the ranks' partial
+// tiles meet through distributed shared memory, each rank summing a share of
+// the columns; whole waves of tiles and the leftover tiles may go to two
+// launches, the leftovers split):
 //   warp 0      TMA producer: x tiles (bf16, 128-byte swizzled, 256 x 64) and
 //               packed code tiles (256 rows x 128 codes, unswizzled) into two
 //               shared-memory rings;
