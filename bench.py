@@ -553,6 +553,32 @@ def oracle_sample(seconds_target=8.0, max_rows=None):
                     f"{tot_t:.2f} s of CPU time")
 
 
+def oracle_quantize_sample(seconds_target=2.0):
+    """The CPU oracle's quantiser (fp64 RTN on every host thread, then its
+    packer) on the first rows of each projection of the 3-bit layer, the
+    workload of the GPU quantiser line; GB/s of fp16 weights read plus codes,
+    scales and zeros written.  Returns (GB/s, description)."""
+    import oracle
+    w = wq_inputs.WORKLOADS[LAYER3B]
+    nthreads = os.cpu_count() or 1
+    R = 64
+    while True:
+        tb, tt = 0, 0.0
+        for li, (name, N, K) in enumerate(w["linears"]):
+            rows = np.arange(min(R, N))
+            Wb = wq_inputs.f16_bits(wq_inputs.weight_f16(0, 900 + li, N, K, dist=w["dist"], rows=rows))
+            t0 = time.perf_counter()
+            q, s, z = oracle.quantize_rtn(Wb, w["bits"], w["group"], nthreads=nthreads)
+            oracle.pack(q, w["bits"])
+            tt += time.perf_counter() - t0
+            n = len(rows)
+            tb += n * K * 2 + n * K * w["bits"] // 8 + n * groups(K, w["group"]) * 4
+        if tt >= seconds_target or all(R >= N for _, N, _ in w["linears"]):
+            return (tb / tt / 1e9, f"oracle fp64 quantise + pack of the first {R} rows of each projection "
+                                   f"of the 3-bit layer, {tt:.2f} s of CPU time")
+        R *= 2
+
+
 def cpu_model():
     try:
         for line in open("/proc/cpuinfo"):
@@ -701,8 +727,9 @@ def run_ours(args, rank, world, local):
     cpu = None
     if not args.no_cpu_baseline and world == 1:
         v, cores, desc = oracle_sample()
+        qv, qdesc = oracle_quantize_sample()
         cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc,
-               "cpu": cpu_model()}
+               "cpu": cpu_model(), "quantize": {"GBps": qv, "sample": qdesc}}
     per_rank = value / world
     nlaunch = 1 + (len(w["linears"]) + 127) // 128
     line = {
