@@ -316,6 +316,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   bool ep_ok = false;                         // dequant warps: accumulators are final
+  // A second launch of this kernel over other tiles of the same y (the
+  // leftover tiles of a two-launch plan) may take SMs as this one frees them.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -594,6 +597,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
   }
+  // Such a second launch ends only after the first has (a no-op otherwise),
+  // so work queued behind it on the stream sees every tile of y.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 // ------------------------------------------------------------------ host
@@ -699,25 +705,31 @@ cudaError_t launch_bits(const __nv_bfloat16* x, int64_t M, int64_t N, int64_t K,
       ks_rest = c;
     }
   }
-  auto launch = [&](int tile0, int count, int ks) -> cudaError_t {
+  // The second of two launches is a programmatic dependent of the first: it
+  // reads only x and the codes and writes other tiles of y, so its CTAs may
+  // start on SMs that the first launch's CTAs leave, and its prologue and
+  // launch latency overlap the first launch's last tiles.
+  auto launch = [&](int tile0, int count, int ks, bool overlap) -> cudaError_t {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(unsigned(count), 1, unsigned(ks));
     cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 1;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = unsigned(ks);
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = overlap ? 2 : 1;
     return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BITS>, tx, tc, scales, zeros, M, N, K, g,
                               FastDiv(uint32_t(g / 32)), y, tile0, ntn);
   };
-  if (whole == 0) return launch(0, tiles, ks_one);
-  cudaError_t e = launch(0, whole, 1);
-  if (e == cudaSuccess) e = launch(whole, tiles - whole, ks_rest);
+  if (whole == 0) return launch(0, tiles, ks_one, false);
+  cudaError_t e = launch(0, whole, 1, false);
+  if (e == cudaSuccess) e = launch(whole, tiles - whole, ks_rest, true);
   return e;
 }
 
