@@ -11,10 +11,11 @@
 // of it when K is split over a thread-block cluster: the ranks' partial
 // tiles meet through distributed shared memory, each rank summing a share of
 // the columns; whole waves of tiles and the leftover tiles may go to two
-// launches, the leftovers split):
+// launches, the leftovers split, the second a programmatic dependent of the
+// first so that it fills SMs as they free up):
 //   warp 0      TMA producer: x tiles (bf16, 128-byte swizzled, 256 x 64) and
 //               packed code tiles (256 rows x 128 codes, unswizzled) into two
-//               shared-memory rings;
+//               shared-memory rings (W' has a third, written by warps 2..9);
 //   warp 1      owns tensor memory (512 columns: two 128 x 256 fp32
 //               accumulators) and one lane issues the MMAs:
 //               tcgen05.mma.cta_group::1.kind::f16, M = 128, N = 256, K = 16,
