@@ -105,3 +105,28 @@ def test_tc_whole_waves_then_split_rest(bits, group):
     oc, os_, oz = oracle_quantize(Wh[cols], bits, group)
     y_ref, bound = oracle.gemm(wq_inputs.bf16_bits(x[torch.from_numpy(rows)]), oc, os_, oz, len(cols), K, bits, group)
     assert_y_close(y[np.ix_(rows, cols)], y_ref, bound, f"152 tiles bits={bits} g={group}")
+
+
+def test_tc_two_launches_keep_stream_order():
+    """With 152 tiles the GEMM runs as a launch of 148 whole tiles and a
+    dependent launch of the 4 left over, which may start before the first
+    ends.  Work queued right behind the GEMM on its stream (here a copy of y)
+    must still see every tile of both launches."""
+    M, N, K, bits, group = 2048, 4864, 2048, 4, 128
+    m = wq()
+    Wh = wq_inputs.weight_f16(32, 0, N, K)
+    x = wq_inputs.activations_bf16(32, 1, M, K).cuda()
+    codes, s, z = m.wq_quantize_rtn(to_dev_f16(Wh), bits, group)
+    ref = m.wq_gemm(x, codes, s, z, bits, group, N, K)
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    for _ in range(3):
+        y = torch.zeros(M, N, dtype=torch.bfloat16, device="cuda")
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            m.wq_gemm(x, codes, s, z, bits, group, N, K, y=y, stream=side)
+            snap = y.clone()
+        side.synchronize()
+        assert m.wq_last_device_error() == m.WQ_OK
+        assert torch.equal(snap, ref)
+        assert torch.equal(y, ref)
