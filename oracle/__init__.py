@@ -19,6 +19,12 @@ Parity status of each function (what pins it, see ``tests/test_oracle.py``):
   round trips).
 * ``dequant`` / ``gemm``: pinned (exact rational sums on tiny inputs, one-hot
   and zero inputs, permutation invariance).
+* ``hessian`` / ``quantize_optq``: pinned (``tests/test_oracle_optq.py``): the
+  compensated weights at every step against the least-squares re-fit solved by
+  ``numpy.linalg.solve``; a diagonal Hessian reproduces ``quantize_rtn`` bit for
+  bit; a factor 4 on H changes nothing; the first column of every row and the
+  first group's grid equal round-to-nearest's; the layer's output error on the
+  calibration rows falls below round-to-nearest's.
 """
 from __future__ import annotations
 
@@ -46,6 +52,9 @@ def _lib():
         lib.orc_quantize_rtn.restype = ctypes.c_int
         lib.orc_quantize_rtn_sym.argtypes = [_p, _i64, _i64, ctypes.c_int, _i64, _p, _p, ctypes.c_int]
         lib.orc_quantize_rtn_sym.restype = ctypes.c_int
+        lib.orc_quantize_optq.argtypes = [_p, _p, _i64, _i64, ctypes.c_int, _i64, ctypes.c_double,
+                                          _p, _p, _p, _p, ctypes.c_int]
+        lib.orc_quantize_optq.restype = ctypes.c_int
         lib.orc_pack.argtypes = [_p, _i64, _i64, ctypes.c_int, _p]
         lib.orc_pack.restype = ctypes.c_int
         lib.orc_unpack.argtypes = [_p, _i64, _i64, ctypes.c_int, _p]
@@ -136,6 +145,41 @@ def quantize_rtn_sym(W_bits, bits: int, group: int, nthreads: int = 0):
     if rc != 0:
         raise OracleError(f"invalid arguments N={N} K={K} bits={bits} group={group}")
     return q, s
+
+
+def hessian(x_bits):
+    """Layer Hessian of calibration activations (reading O1 of the C++
+    source): ``H = (2 / S) X^T X`` in fp64 for bf16 bit patterns ``x_bits``
+    [S, K]."""
+    X = bf16_to_f64(x_bits)
+    return (2.0 / X.shape[0]) * (X.T @ X)
+
+
+def quantize_optq(W_bits, H, bits: int, group: int, percdamp: float = 0.01,
+                  return_u: bool = False, nthreads: int = 0):
+    """Error-compensating quantisation of fp16 ``W`` (uint16 bit patterns
+    [N, K]) against the layer Hessian ``H`` (fp64 [K, K]).
+
+    Returns ``(q, scales, zeros)`` like ``quantize_rtn`` and, with
+    ``return_u``, the fp64 weights [N, K] as each column came up."""
+    W = _c(W_bits, np.uint16)
+    N, K = W.shape
+    Hc = _c(H, np.float64)
+    if Hc.shape != (K, K):
+        raise OracleError("H must be [K, K]")
+    G = 1 if group in (0, K) else (K // group if group > 0 and K % group == 0 else 1)
+    q = np.empty((N, K), np.uint8)
+    s = np.empty((N, G), np.uint16)
+    z = np.empty((N, G), np.uint16)
+    u = np.empty((N, K), np.float64) if return_u else None
+    rc = _lib().orc_quantize_optq(_ptr(W), _ptr(Hc), N, K, bits, group, float(percdamp),
+                                  _ptr(q), _ptr(s), _ptr(z), _ptr(u) if return_u else None,
+                                  nthreads)
+    if rc == -2:
+        raise OracleError("the damped Hessian is not positive definite")
+    if rc != 0:
+        raise OracleError(f"invalid arguments N={N} K={K} bits={bits} group={group}")
+    return (q, s, z, u) if return_u else (q, s, z)
 
 
 def sym_zeros(scales, bits: int):

@@ -47,6 +47,29 @@
 //      u = k/32 fill the 96-bit little-endian value of words 3u..3u+2, code
 //      j = k mod 32 at bit 3j (codes 10 and 21 straddle two words).
 //
+//   * Error-compensating quantisation (OPTQ).  "OPTQ: Accurate Quantization
+//     for Generative Pre-trained Transformers" (reproducibility summary, rows
+//     "Experiment Setup" and "Pseudocode") and "Platform For AI: BladeLLM model
+//     quantization", "Quantization algorithms > GPTQ": the columns of a row are
+//     quantised one after another; after each, the error it leaves is made up
+//     by adjusting the columns not yet quantised through the inverse of the
+//     layer Hessian of the calibration activations.  Readings:
+//   O1 the Hessian is H = (2 / S) X^T X over S calibration rows x (any positive
+//      factor gives the same codes: it cancels, damping included);
+//   O2 damping: H + d I with d = percdamp * mean(diag H) (percdamp 0.01 by
+//      default); if every diagonal entry is 0, H is replaced by I;
+//   O3 a group's grid (R1-R5) is computed from the compensated weights of the
+//      whole group when its first column comes up, and then stays fixed;
+//   O4 columns are taken in their natural order; the grid rules apply to the
+//      fp64 compensated weights as they are (no rounding to fp16 first);
+//   O5 each step's compensation is the least-squares re-fit: after columns
+//      0..k are fixed to their grid values w', the free columns F = k+1..K-1
+//      become w0_F - H_FF^-1 H_F,Q (w'_Q - w0_Q) (Q = 0..k, w0 the fp16
+//      weights, H damped).  Carried out step by step this is
+//        e = (w_k - w'_k) / A_kk;  w_j -= e A_kj  (j > k)
+//      with A the inverse of H restricted to the columns free before step k;
+//      A is then reduced by eliminating column k.
+//
 // Everything is computed in fp64.  fp16 and bf16 are decoded and rounded here
 // from the IEEE 754 binary16 / bfloat16 definitions (no library conversion).
 
@@ -270,6 +293,116 @@ int orc_quantize_rtn_sym(const uint16_t* W, int64_t N, int64_t K, int bits, int6
         c = std::min(std::max(c, 0.0), qmax);
         q[n * K + k] = uint8_t(c);
       }
+    }
+  });
+  return 0;
+}
+
+// ------------------------------------------------ quantise with error compensation (OPTQ)
+// W: fp16 bit patterns [N, K]; H: fp64 [K, K], symmetric positive
+// semi-definite (only its lower triangle is read).  Outputs as for
+// orc_quantize_rtn; u (optional, fp64 [N, K]) receives each weight as it was
+// when its column came up (after the compensation of the earlier columns).
+// Returns 0, -1 on an invalid argument, -2 if the damped H is not positive
+// definite (nothing written).
+int orc_quantize_optq(const uint16_t* W, const double* H, int64_t N, int64_t K, int bits,
+                      int64_t group, double percdamp, uint8_t* q, uint16_t* scales,
+                      uint16_t* zeros, double* u, int nthreads) {
+  if (!W || !H || !q || !scales || !zeros || N < 1 || K < 1 || !valid_bits(bits) ||
+      !(percdamp >= 0.0))
+    return -1;
+  const int64_t g = effective_group(K, group);
+  if (g < 0) return -1;
+  const int64_t G = K / g;
+  const double qmax = double((1 << bits) - 1);
+  const size_t KK = size_t(K) * size_t(K);
+
+  // O2: damped Hessian (lower triangle, full storage).
+  std::vector<double> Hd(KK, 0.0);
+  double mean_diag = 0.0;
+  for (int64_t i = 0; i < K; ++i) mean_diag += H[i * K + i];
+  mean_diag /= double(K);
+  for (int64_t i = 0; i < K; ++i)
+    for (int64_t j = 0; j <= i; ++j)
+      Hd[i * K + j] = mean_diag == 0.0 ? (i == j ? 1.0 : 0.0) : H[i * K + j];
+  if (mean_diag != 0.0)
+    for (int64_t i = 0; i < K; ++i) Hd[i * K + i] += percdamp * mean_diag;
+
+  // A = Hd^-1 through the Cholesky factor Hd = L L^T: A = L^-T L^-1.
+  std::vector<double> L(KK, 0.0);
+  for (int64_t j = 0; j < K; ++j) {
+    double d = Hd[j * K + j];
+    for (int64_t p = 0; p < j; ++p) d -= L[j * K + p] * L[j * K + p];
+    if (!(d > 0.0)) return -2;
+    const double ljj = std::sqrt(d);
+    L[j * K + j] = ljj;
+    for (int64_t i = j + 1; i < K; ++i) {
+      double v = Hd[i * K + j];
+      for (int64_t p = 0; p < j; ++p) v -= L[i * K + p] * L[j * K + p];
+      L[i * K + j] = v / ljj;
+    }
+  }
+  std::vector<double> Li(KK, 0.0);   // L^-1, lower triangular
+  for (int64_t c = 0; c < K; ++c) {
+    Li[c * K + c] = 1.0 / L[c * K + c];
+    for (int64_t i = c + 1; i < K; ++i) {
+      double v = 0.0;
+      for (int64_t p = c; p < i; ++p) v -= L[i * K + p] * Li[p * K + c];
+      Li[i * K + c] = v / L[i * K + i];
+    }
+  }
+  std::vector<double> A(KK, 0.0);
+  for (int64_t i = 0; i < K; ++i)
+    for (int64_t j = 0; j < K; ++j) {
+      double v = 0.0;
+      for (int64_t p = std::max(i, j); p < K; ++p) v += Li[p * K + i] * Li[p * K + j];
+      A[i * K + j] = v;
+    }
+
+  // O5: the pivot and the row of A each step uses; A then loses column k.
+  // Every row of W meets the same sequence, so it is recorded once.
+  std::vector<double> piv(static_cast<size_t>(K));
+  std::vector<double> arow(KK, 0.0);   // arow[k*K + j] = A_kj at step k, j > k
+  for (int64_t k = 0; k < K; ++k) {
+    const double akk = A[k * K + k];
+    piv[size_t(k)] = akk;
+    for (int64_t j = k + 1; j < K; ++j) arow[k * K + j] = A[k * K + j];
+    for (int64_t i = k + 1; i < K; ++i) {
+      const double f = A[i * K + k] / akk;
+      for (int64_t j = k + 1; j < K; ++j) A[i * K + j] -= f * A[k * K + j];
+    }
+  }
+
+  parallel_rows(N, nthreads, [&](int64_t n) {
+    std::vector<double> w(static_cast<size_t>(K));
+    for (int64_t k = 0; k < K; ++k) w[size_t(k)] = f16(W[n * K + k]);
+    double s = 1.0, z = 0.0;
+    for (int64_t k = 0; k < K; ++k) {
+      if (k % g == 0) {
+        // O3: the group's grid from its current (compensated) weights, R1-R5.
+        const int64_t j = k / g;
+        double lo = 0.0, hi = 0.0;
+        for (int64_t c = k; c < k + g; ++c) {
+          lo = std::min(lo, w[size_t(c)]);
+          hi = std::max(hi, w[size_t(c)]);
+        }
+        s = f16(to_f16((hi - lo) / qmax));
+        if (s == 0.0) {
+          s = 1.0;
+          z = 0.0;
+        } else {
+          z = std::nearbyint((0.0 - lo) / s);
+        }
+        scales[n * G + j] = to_f16(s);
+        zeros[n * G + j] = to_f16(z);
+      }
+      const double wk = w[size_t(k)];
+      if (u) u[n * K + k] = wk;
+      double c = std::nearbyint(wk / s) + z;
+      c = std::min(std::max(c, 0.0), qmax);
+      q[n * K + k] = uint8_t(c);
+      const double e = (wk - s * (c - z)) / piv[size_t(k)];
+      for (int64_t j = k + 1; j < K; ++j) w[size_t(j)] -= e * arow[k * K + j];
     }
   });
   return 0;

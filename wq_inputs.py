@@ -1,7 +1,8 @@
 """Seeded synthetic inputs shared by the oracle checks and the CUDA path.
 
-This module holds no quantisation or matmul arithmetic: it only draws random
-numbers and casts them to the storage types (fp16 weights, bf16 activations),
+This module holds none of the method's arithmetic: it only draws random
+numbers (mixing latent factors into correlated features for the calibration
+rows) and casts them to the storage types (fp16 weights, bf16 activations),
 so the oracle (``oracle/``) and the library (``quantized_gemm_wq_b200``) are
 handed the very same bytes.
 
@@ -18,6 +19,15 @@ in for real checkpoints):
 * activations ``x`` bf16 ``[M, K]``: ``N(0, 1)`` drawn in float32 per row
   stream ``(seed, tensor_id, 1_000_000 + m)`` and rounded to bf16 by torch's
   CPU cast (round-to-nearest-even).
+
+* calibration activations bf16 ``[S, K]`` (stand-in for the pages' 128
+  segments of 2048 tokens of C4 text): correlated features with a few
+  outlier channels, ``x = c * (z + lam @ f)`` with ``z ~ N(0, I_K)``,
+  ``RANK`` latent factors ``f ~ N(0, I)`` per row, loadings
+  ``lam ~ N(0, 1/RANK)`` per feature, and per-feature scales ``c`` = 1 except
+  ``OUTLIER_FRAC`` of the features at ``OUTLIER_SCALE``; drawn in float64 from
+  one stream keyed by ``(seed, tensor_id, 2_000_000)``, rounded to bf16 by
+  torch's CPU cast.
 
 The workload table ``WORKLOADS`` lists the five single-GPU configurations the
 library is tested and measured on (shapes of a single 4096x4096 linear, a
@@ -68,6 +78,24 @@ def activations_bf16(seed: int, tensor_id: int, M: int, K: int) -> torch.Tensor:
     for m in range(M):
         g = np.random.default_rng([int(seed), int(tensor_id), 1_000_000 + m])
         v[m] = g.standard_normal(K, dtype=np.float32)
+    return torch.from_numpy(v).to(torch.bfloat16)
+
+
+CALIB_RANK = 16
+CALIB_OUTLIER_FRAC = 0.02
+CALIB_OUTLIER_SCALE = 20.0
+
+
+def calibration_bf16(seed: int, tensor_id: int, S: int, K: int) -> torch.Tensor:
+    """bf16 calibration activations ``[S, K]`` on the CPU (recipe above)."""
+    g = np.random.default_rng([int(seed), int(tensor_id), 2_000_000])
+    lam = g.standard_normal((CALIB_RANK, K)) / np.sqrt(CALIB_RANK)
+    c = np.ones(K)
+    n_out = max(1, int(round(CALIB_OUTLIER_FRAC * K)))
+    c[g.choice(K, n_out, replace=False)] = CALIB_OUTLIER_SCALE
+    f = g.standard_normal((S, CALIB_RANK))
+    z = g.standard_normal((S, K))
+    v = (z + f @ lam) * c
     return torch.from_numpy(v).to(torch.bfloat16)
 
 
